@@ -1,0 +1,619 @@
+// C ABI of the Q4_0 decode library: argument checks (before any CUDA call),
+// launch planning, the layer stack with programmatic dependent launch, CUDA
+// graph capture, host interchange helpers and the host-side plan validator.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/q4.h"
+#include "../../include/q4_debug.h"
+#include "q4_device.cuh"
+#include "q4_plan.h"
+
+namespace q4k {
+cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblocks,
+                        cudaStream_t stream);
+cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int64_t nblocks,
+                           cudaStream_t stream);
+cudaError_t setup_gemv_kernels();
+cudaError_t launch_gemv(const q4plan::GemvParams& P, bool pdl, cudaStream_t stream);
+}  // namespace q4k
+
+using q4plan::GemvDesc;
+using q4plan::GemvParams;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// CTAs a launch aims for before K is split further: two per SM of a B200.
+constexpr int64_t kTargetUnits = 2 * 148;
+constexpr int kMaxCudaCoreBatch = 4;
+constexpr uint32_t kMaxSmem = 227 * 1024;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+q4_status check_shape(int64_t n, int64_t k) {
+    if (n < 1 || k < Q4_QK || k % Q4_QK != 0) return Q4_ERR_INVALID_ARG;
+    if (n > (int64_t(1) << 34) || k > (int64_t(1) << 34)) return Q4_ERR_INVALID_ARG;
+    return Q4_OK;
+}
+
+q4_status check_matrix(const q4_matrix* m) {
+    if (!m || !m->qs || !m->d) return Q4_ERR_INVALID_ARG;
+    q4_status s = check_shape(m->n, m->k);
+    if (s != Q4_OK) return s;
+    if (!aligned(m->qs, 16) || !aligned(m->d, 16)) return Q4_ERR_MISALIGNED;
+    return Q4_OK;
+}
+
+struct Shape {
+    int64_t n, k;
+};
+
+// Plan one launch over `count` GEMVs of the given shapes. Fills everything in P
+// except the pointers, and the workspace bytes it needs.
+q4_status plan_shapes(const Shape* sh, int count, int batch, GemvParams* P, size_t* ws_bytes) {
+    if (count < 1 || count > Q4_MAX_GROUP || batch < 1 || batch > kMaxCudaCoreBatch)
+        return Q4_ERR_INVALID_ARG;
+    std::memset(P, 0, sizeof *P);
+    const int maxb = q4plan::max_blocks_per_split(batch);
+    int64_t base_units = 0;
+    for (int i = 0; i < count; ++i) {
+        q4_status s = check_shape(sh[i].n, sh[i].k);
+        if (s != Q4_OK) return s;
+        base_units += ceil_div(sh[i].n, q4plan::kRowsPerCta) * ceil_div(sh[i].k / Q4_QK, maxb);
+    }
+    const int64_t factor = base_units >= kTargetUnits ? 1 : ceil_div(kTargetUnits, base_units);
+    int64_t units = 0;
+    int64_t off = q4plan::kHeaderBytes;
+    int nbs_max = 1;
+    for (int i = 0; i < count; ++i) {
+        GemvDesc& G = P->g[i];
+        const int64_t nb = sh[i].k / Q4_QK;
+        const int64_t tiles = ceil_div(sh[i].n, q4plan::kRowsPerCta);
+        const int64_t smin = ceil_div(nb, maxb);
+        int64_t S = smin * factor;
+        S = std::min(S, std::max(smin, nb / 8));  // splits keep at least 8 blocks
+        int64_t nbs = ceil_div(nb, S);
+        if (nbs > 8) nbs = std::min<int64_t>(round_up(nbs, 8), maxb);
+        S = ceil_div(nb, nbs);
+        G.n = sh[i].n;
+        G.nb = (int32_t)nb;
+        G.splits = (int32_t)S;
+        G.nb_split = (int32_t)nbs;
+        G.row_tiles = (int32_t)tiles;
+        G.unit_begin = (int32_t)units;
+        if (S > 1) {
+            G.ticket_off = off / 4;
+            off += round_up(tiles * 4, 256);
+            G.part_off = off / 4;
+            off += round_up((int64_t)batch * S * sh[i].n * 4, 256);
+        }
+        units += tiles * S;
+        nbs_max = std::max<int>(nbs_max, (int)nbs);
+        if (units > INT_MAX / 2) return Q4_ERR_INVALID_ARG;
+    }
+    P->count = count;
+    P->total_units = (int32_t)units;
+    P->batch = batch;
+    if (batch == 1)
+        P->smem_x = (uint32_t)ceil_div(nbs_max, 32) * 32 * 8 * 16;
+    else
+        P->smem_x = (uint32_t)(batch * q4plan::x_token_slots_bs(nbs_max) * 16);
+    P->smem_qs_warp = (uint32_t)(q4plan::kRowsPerWarp * nbs_max * 16);
+    P->d_slot = (uint32_t)round_up(nbs_max + 14, 8);
+    P->smem_d_warp = (uint32_t)(q4plan::kRowsPerWarp * P->d_slot * 2);
+    P->smem_total = q4plan::kBarrierBytes + P->smem_x +
+                    q4plan::kWarps * (P->smem_qs_warp + P->smem_d_warp);
+    if (P->smem_total > kMaxSmem) return Q4_ERR_UNSUPPORTED;
+    *ws_bytes = (size_t)off;
+    return Q4_OK;
+}
+
+// Token chunks: batches above the CUDA-core kernel's width run as several
+// launches of at most kMaxCudaCoreBatch tokens.
+int chunk_tokens(int b, int c0) { return std::min(kMaxCudaCoreBatch, b - c0); }
+
+std::mutex g_dev_mu;
+bool g_dev_ready[64];
+
+q4_status ensure_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return Q4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return Q4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_dev_ready[dev]) return Q4_OK;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    if (major != 10 || minor != 0) return Q4_ERR_UNSUPPORTED;
+    if (q4k::setup_gemv_kernels() != cudaSuccess) return Q4_ERR_CUDA;
+    g_dev_ready[dev] = true;
+    return Q4_OK;
+}
+
+struct GemvCall {
+    q4_matrix m;
+    const float* x;
+    float* y;
+};
+
+// Validate and plan one group for `b` tokens; returns the workspace bytes needed.
+q4_status check_group(const GemvCall* calls, int count, int b, size_t* ws_need) {
+    if (count < 1 || count > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
+    if (b < 1 || b > Q4_MAX_BATCH) return Q4_ERR_UNSUPPORTED;
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+        q4_status s = check_matrix(&calls[i].m);
+        if (s != Q4_OK) return s;
+        if (!calls[i].x || !calls[i].y) return Q4_ERR_INVALID_ARG;
+        if (!aligned(calls[i].x, 16) || !aligned(calls[i].y, 16)) return Q4_ERR_MISALIGNED;
+        sh[i] = {calls[i].m.n, calls[i].m.k};
+    }
+    size_t need = 0;
+    for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
+        GemvParams P;
+        size_t w = 0;
+        q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), &P, &w);
+        if (s != Q4_OK) return s;
+        need = std::max(need, w);
+    }
+    *ws_need = need;
+    return Q4_OK;
+}
+
+q4_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (!ws || ws_bytes < need) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_MISALIGNED;
+    return Q4_OK;
+}
+
+// Enqueue one group (all token chunks). The first launch may use PDL only if
+// `pdl_first` is set.
+q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, bool pdl_first,
+                       cudaStream_t stream) {
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) sh[i] = {calls[i].m.n, calls[i].m.k};
+    bool pdl = pdl_first;
+    for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
+        const int bt = chunk_tokens(b, c0);
+        GemvParams P;
+        size_t w = 0;
+        q4_status s = plan_shapes(sh, count, bt, &P, &w);
+        if (s != Q4_OK) return s;
+        for (int i = 0; i < count; ++i) {
+            P.g[i].qs = calls[i].m.qs;
+            P.g[i].d = calls[i].m.d;
+            P.g[i].x = calls[i].x + (int64_t)c0 * calls[i].m.k;
+            P.g[i].y = calls[i].y + (int64_t)c0 * calls[i].m.n;
+        }
+        P.ws = static_cast<uint32_t*>(ws);
+        if (q4k::launch_gemv(P, pdl, stream) != cudaSuccess) return Q4_ERR_CUDA;
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        pdl = true;
+    }
+    return Q4_OK;
+}
+
+// Split a stack into groups: [begin, end) index ranges.
+q4_status stack_groups(const q4_stack* s, std::vector<std::pair<int, int>>* out) {
+    if (!s || s->count < 1 || !s->mats || !s->x || !s->y || !s->group) return Q4_ERR_INVALID_ARG;
+    out->clear();
+    int begin = 0;
+    for (int i = 1; i <= s->count; ++i) {
+        if (i < s->count && s->group[i] < s->group[i - 1]) return Q4_ERR_INVALID_ARG;
+        if (i == s->count || s->group[i] != s->group[i - 1]) {
+            if (i - begin > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
+            out->push_back({begin, i});
+            begin = i;
+        }
+    }
+    return Q4_OK;
+}
+
+q4_status stack_check(const q4_stack* s, int b, std::vector<std::pair<int, int>>* groups,
+                      size_t* need) {
+    q4_status st = stack_groups(s, groups);
+    if (st != Q4_OK) return st;
+    size_t mx = 0;
+    for (auto& g : *groups) {
+        GemvCall calls[Q4_MAX_GROUP];
+        for (int i = g.first; i < g.second; ++i)
+            calls[i - g.first] = {s->mats[i], s->x[i], s->y[i]};
+        size_t w = 0;
+        st = check_group(calls, g.second - g.first, b, &w);
+        if (st != Q4_OK) return st;
+        mx = std::max(mx, w);
+    }
+    *need = mx;
+    return Q4_OK;
+}
+
+uint64_t stack_kernel_count(const std::vector<std::pair<int, int>>& groups, int b) {
+    return (uint64_t)groups.size() * (uint64_t)ceil_div(b, kMaxCudaCoreBatch);
+}
+
+}  // namespace
+
+struct q4_graph_s {
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    uint64_t kernels;
+};
+
+extern "C" {
+
+q4_status q4_plane_bytes(int64_t n, int64_t k, size_t* qs_bytes, size_t* d_bytes) {
+    if (check_shape(n, k) != Q4_OK || !qs_bytes || !d_bytes) return Q4_ERR_INVALID_ARG;
+    *qs_bytes = (size_t)(n * (k / 2));
+    *d_bytes = (size_t)round_up(n * (k / Q4_QK) * 2, 16);
+    return Q4_OK;
+}
+
+q4_status q4_pack(const float* w, const q4_matrix* out, void* stream) {
+    q4_status s = check_matrix(out);
+    if (s != Q4_OK) return s;
+    if (!w) return Q4_ERR_INVALID_ARG;
+    if (!aligned(w, 16)) return Q4_ERR_MISALIGNED;
+    if ((s = ensure_device()) != Q4_OK) return s;
+    const int64_t nblocks = out->n * (out->k / Q4_QK);
+    if (q4k::launch_pack(w, out->qs, out->d, nblocks, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return Q4_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return Q4_OK;
+}
+
+q4_status q4_dequant(const q4_matrix* m, float* w_out, void* stream) {
+    q4_status s = check_matrix(m);
+    if (s != Q4_OK) return s;
+    if (!w_out) return Q4_ERR_INVALID_ARG;
+    if (!aligned(w_out, 16)) return Q4_ERR_MISALIGNED;
+    if ((s = ensure_device()) != Q4_OK) return s;
+    const int64_t nblocks = m->n * (m->k / Q4_QK);
+    if (q4k::launch_dequant(m->qs, m->d, w_out, nblocks, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return Q4_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return Q4_OK;
+}
+
+size_t q4_workspace_bytes(int64_t n, int64_t k, int b) {
+    if (check_shape(n, k) != Q4_OK || b < 1 || b > Q4_MAX_BATCH) return 0;
+    size_t need = 0;
+    const Shape sh = {n, k};
+    for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
+        GemvParams P;
+        size_t w = 0;
+        if (plan_shapes(&sh, 1, chunk_tokens(b, c0), &P, &w) != Q4_OK) return 0;
+        need = std::max(need, w);
+    }
+    return need;
+}
+
+q4_status q4_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes < (size_t)q4plan::kHeaderBytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_MISALIGNED;
+    if (cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    return Q4_OK;
+}
+
+q4_status q4_workspace_status(const void* ws, void* stream) {
+    if (!ws) return Q4_ERR_WORKSPACE;
+    uint32_t flag = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&flag, ws, sizeof flag, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return Q4_ERR_CUDA;
+    return flag ? Q4_ERR_TIMEOUT : Q4_OK;
+}
+
+q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, void* ws,
+                          size_t ws_bytes, void* stream) {
+    if (!m) return Q4_ERR_INVALID_ARG;
+    GemvCall call = {*m, X, Y};
+    size_t need = 0;
+    q4_status s = check_group(&call, 1, b, &need);
+    if (s != Q4_OK) return s;
+    if ((s = check_ws(ws, ws_bytes, need)) != Q4_OK) return s;
+    if ((s = ensure_device()) != Q4_OK) return s;
+    return launch_group(&call, 1, b, ws, false, static_cast<cudaStream_t>(stream));
+}
+
+q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t ws_bytes,
+                  void* stream) {
+    return q4_gemv_batched(m, x, 1, y, ws, ws_bytes, stream);
+}
+
+size_t q4_stack_workspace_bytes(const q4_stack* s, int b) {
+    std::vector<std::pair<int, int>> groups;
+    size_t need = 0;
+    if (stack_check(s, b, &groups, &need) != Q4_OK) return 0;
+    return need;
+}
+
+q4_status q4_layer_stack(const q4_stack* s, int b, void* ws, size_t ws_bytes, void* stream) {
+    std::vector<std::pair<int, int>> groups;
+    size_t need = 0;
+    q4_status st = stack_check(s, b, &groups, &need);
+    if (st != Q4_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, need)) != Q4_OK) return st;
+    if ((st = ensure_device()) != Q4_OK) return st;
+    bool first = true;
+    for (auto& g : groups) {
+        GemvCall calls[Q4_MAX_GROUP];
+        for (int i = g.first; i < g.second; ++i)
+            calls[i - g.first] = {s->mats[i], s->x[i], s->y[i]};
+        st = launch_group(calls, g.second - g.first, b, ws, !first,
+                          static_cast<cudaStream_t>(stream));
+        if (st != Q4_OK) return st;
+        first = false;
+    }
+    return Q4_OK;
+}
+
+q4_status q4_stack_graph_create(const q4_stack* s, int b, void* ws, size_t ws_bytes, void* stream,
+                                q4_graph* out) {
+    if (!out || !stream) return Q4_ERR_INVALID_ARG;
+    *out = nullptr;
+    std::vector<std::pair<int, int>> groups;
+    size_t need = 0;
+    q4_status st = stack_check(s, b, &groups, &need);
+    if (st != Q4_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, need)) != Q4_OK) return st;
+    if ((st = ensure_device()) != Q4_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(cs, &cap) != cudaSuccess) return Q4_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return Q4_ERR_INVALID_ARG;
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    const uint64_t before = g_launches.load();
+    q4_status run = q4_layer_stack(s, b, ws, ws_bytes, stream);
+    g_launches.store(before);  // captured launches do not run now
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(cs, &graph);
+    if (run != Q4_OK || e != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        return run != Q4_OK ? run : Q4_ERR_CUDA;
+    }
+    cudaGraphExec_t exec = nullptr;
+    if (cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+        cudaGraphDestroy(graph);
+        return Q4_ERR_CUDA;
+    }
+    q4_graph g = new (std::nothrow) q4_graph_s;
+    if (!g) {
+        cudaGraphExecDestroy(exec);
+        cudaGraphDestroy(graph);
+        return Q4_ERR_INVALID_ARG;
+    }
+    g->graph = graph;
+    g->exec = exec;
+    g->kernels = stack_kernel_count(groups, b);
+    *out = g;
+    return Q4_OK;
+}
+
+q4_status q4_graph_launch(q4_graph g, void* stream) {
+    if (!g) return Q4_ERR_INVALID_ARG;
+    if (cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    g_launches.fetch_add(g->kernels, std::memory_order_relaxed);
+    return Q4_OK;
+}
+
+q4_status q4_graph_destroy(q4_graph g) {
+    if (!g) return Q4_ERR_INVALID_ARG;
+    cudaError_t e1 = cudaGraphExecDestroy(g->exec);
+    cudaError_t e2 = cudaGraphDestroy(g->graph);
+    delete g;
+    return (e1 == cudaSuccess && e2 == cudaSuccess) ? Q4_OK : Q4_ERR_CUDA;
+}
+
+q4_status q4_blocks_to_planes(const uint8_t* blocks, int64_t n, int64_t k, uint8_t* qs,
+                              uint16_t* d) {
+    if (!blocks || !qs || !d || check_shape(n, k) != Q4_OK) return Q4_ERR_INVALID_ARG;
+    const int64_t nblocks = n * (k / Q4_QK);
+    for (int64_t i = 0; i < nblocks; ++i) {
+        const uint8_t* b = blocks + i * Q4_BLOCK_BYTES;
+        d[i] = (uint16_t)(b[0] | (b[1] << 8));
+        std::memcpy(qs + i * 16, b + 2, 16);
+    }
+    return Q4_OK;
+}
+
+q4_status q4_planes_to_blocks(const uint8_t* qs, const uint16_t* d, int64_t n, int64_t k,
+                              uint8_t* blocks) {
+    if (!blocks || !qs || !d || check_shape(n, k) != Q4_OK) return Q4_ERR_INVALID_ARG;
+    const int64_t nblocks = n * (k / Q4_QK);
+    for (int64_t i = 0; i < nblocks; ++i) {
+        uint8_t* b = blocks + i * Q4_BLOCK_BYTES;
+        b[0] = (uint8_t)(d[i] & 0xFF);
+        b[1] = (uint8_t)(d[i] >> 8);
+        std::memcpy(b + 2, qs + i * 16, 16);
+    }
+    return Q4_OK;
+}
+
+const char* q4_status_string(q4_status s) {
+    switch (s) {
+        case Q4_OK: return "ok";
+        case Q4_ERR_INVALID_ARG: return "invalid argument";
+        case Q4_ERR_MISALIGNED: return "misaligned pointer";
+        case Q4_ERR_WORKSPACE: return "workspace missing or too small";
+        case Q4_ERR_UNSUPPORTED: return "unsupported (batch or device)";
+        case Q4_ERR_CUDA: return "CUDA error";
+        case Q4_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+uint64_t q4_launch_count(void) { return g_launches.load(); }
+
+// ---------------------------------------------------------------------------
+// host-side diagnostics
+// ---------------------------------------------------------------------------
+
+q4_status q4_debug_plan_info(const int64_t* n, const int64_t* k, int count, int b, int64_t* out) {
+    if (!n || !k || !out || count < 1 || count > Q4_MAX_GROUP || b < 1 || b > kMaxCudaCoreBatch)
+        return Q4_ERR_INVALID_ARG;
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
+    GemvParams P;
+    size_t w = 0;
+    q4_status s = plan_shapes(sh, count, b, &P, &w);
+    if (s != Q4_OK) return s;
+    out[0] = P.total_units;
+    out[1] = P.smem_total;
+    out[2] = (int64_t)w;
+    for (int i = 0; i < count; ++i) out[3 + i] = P.g[i].splits;
+    return Q4_OK;
+}
+
+int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b) {
+    using namespace q4plan;
+    if (!n || !k || count < 1 || count > Q4_MAX_GROUP || b < 1 || b > kMaxCudaCoreBatch) return 1;
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
+    GemvParams P;
+    size_t ws_bytes = 0;
+    if (plan_shapes(sh, count, b, &P, &ws_bytes) != Q4_OK) return 2;
+    if (P.smem_total > kMaxSmem) return 3;
+    if (P.smem_x % 16 || P.smem_qs_warp % 16 || P.smem_d_warp % 16) return 4;
+    if ((int64_t)kBarrierBytes < (int64_t)kWarps * 8) return 5;
+    std::vector<std::vector<uint8_t>> cover(count);
+    for (int i = 0; i < count; ++i) cover[i].assign((size_t)(sh[i].n * (sh[i].k / Q4_QK)), 0);
+    int64_t units_seen = 0;
+    for (int unit = 0; unit < P.total_units; ++unit) {
+        const Unit u = unit_of(P, unit);
+        if (u.g < 0 || u.g >= count) return 10;
+        const GemvDesc& G = P.g[u.g];
+        if (u.tile < 0 || u.tile >= G.row_tiles || u.split < 0 || u.split >= G.splits) return 11;
+        const int kbs = split_blocks(G, u.split);
+        if (kbs < 1 || kbs > G.nb_split) return 12;
+        const int64_t qs_plane = sh[u.g].n * (sh[u.g].k / 2);
+        const int64_t d_plane = round_up(sh[u.g].n * G.nb * 2, 16);
+        // activations of the split
+        const int64_t x0 = (int64_t)u.split * G.nb_split * 32;
+        if (x0 + (int64_t)kbs * 32 > sh[u.g].k) return 13;
+        if (b == 1) {
+            for (int j = 0; j < kbs; ++j)
+                for (int c = 0; c < 8; ++c)
+                    if ((int64_t)(x_slot_b1(j, c) + 1) * 16 > P.smem_x) return 14;
+        } else {
+            const int slots = x_token_slots_bs(G.nb_split);
+            for (int j = 0; j < kbs; ++j)
+                for (int c = 0; c < 8; ++c)
+                    if (x_slot_bs(j, c) >= slots || (int64_t)(b * slots) * 16 > P.smem_x) return 15;
+        }
+        for (int warp = 0; warp < kWarps; ++warp) {
+            const int rows = warp_rows(G, u.tile, warp);
+            const int64_t row0 = (int64_t)u.tile * kRowsPerCta + (int64_t)warp * kRowsPerWarp;
+            const int64_t wbase = smem_warp_offset(P, warp);
+            if (wbase % 16) return 16;
+            if (wbase + P.smem_qs_warp + P.smem_d_warp > P.smem_total) return 17;
+            int64_t tx = 0;
+            for (int r = 0; r < rows; ++r) {
+                const int64_t row = row0 + r;
+                if (row >= sh[u.g].n) return 18;
+                const int64_t qsrc = qs_src_offset(G, row, u.split);
+                if (qsrc < 0 || qsrc % 16 || qsrc + (int64_t)kbs * 16 > qs_plane) return 19;
+                const int64_t qdst = (int64_t)r * G.nb_split * 16;
+                if (qdst + (int64_t)kbs * 16 > P.smem_qs_warp) return 20;
+                const DRange dr = d_range(G, row, u.split, kbs);
+                if (dr.src < 0 || dr.src % 16 || dr.bytes % 16 || dr.bytes == 0) return 21;
+                if (dr.src + dr.bytes > d_plane) return 22;
+                if ((int64_t)r * P.d_slot * 2 + dr.bytes > P.smem_d_warp) return 23;
+                if (dr.shift + (uint32_t)kbs > P.d_slot) return 24;
+                if ((int64_t)dr.shift * 2 + (int64_t)kbs * 2 > dr.bytes) return 25;
+                tx += (int64_t)kbs * 16 + dr.bytes;
+                for (int j = 0; j < kbs; ++j) {
+                    uint8_t& c = cover[u.g][(size_t)(row * G.nb + (int64_t)u.split * G.nb_split + j)];
+                    if (c) return 26;
+                    c = 1;
+                }
+            }
+            if (tx >= (int64_t(1) << 20)) return 27;
+        }
+        if (G.splits > 1) {
+            if ((G.ticket_off + G.row_tiles) * 4 > (int64_t)ws_bytes) return 28;
+            if ((G.part_off + (int64_t)b * G.splits * G.n) * 4 > (int64_t)ws_bytes) return 29;
+            if (G.ticket_off * 4 < kHeaderBytes || G.part_off * 4 < kHeaderBytes) return 30;
+        }
+        ++units_seen;
+    }
+    for (int i = 0; i < count; ++i)
+        for (uint8_t c : cover[i])
+            if (!c) return 31;
+    // workspace regions of different GEMVs do not overlap
+    for (int i = 0; i < count; ++i)
+        for (int j = i + 1; j < count; ++j) {
+            const GemvDesc &A = P.g[i], &B = P.g[j];
+            if (A.splits < 2 || B.splits < 2) continue;
+            const int64_t a0 = A.ticket_off * 4, a1 = (A.part_off + (int64_t)b * A.splits * A.n) * 4;
+            const int64_t b0 = B.ticket_off * 4, b1 = (B.part_off + (int64_t)b * B.splits * B.n) * 4;
+            if (a0 < b1 && b0 < a1) return 32;
+        }
+    return units_seen == P.total_units ? 0 : 33;
+}
+
+int64_t q4_debug_check_unpack(uint64_t seed, int64_t count) {
+    int64_t bad = 0;
+    auto check = [&](uint32_t word) {
+        const q4dev::Pairs p = q4dev::unpack_word(word);
+        auto code = [&](int bit) { return (float)((int)((word >> bit) & 0xFu) - 8); };
+        // byte m: low nibble at bit 8m -> weight 4w+m, high nibble at 8m+4 -> 16+4w+m
+        bad += p.lo01.x != code(0);
+        bad += p.lo01.y != code(8);
+        bad += p.lo23.x != code(16);
+        bad += p.lo23.y != code(24);
+        bad += p.hi01.x != code(4);
+        bad += p.hi01.y != code(12);
+        bad += p.hi23.x != code(20);
+        bad += p.hi23.y != code(28);
+    };
+    for (int nib = 0; nib < 8; ++nib)
+        for (uint32_t v = 0; v < 16; ++v) check(v << (4 * nib));
+    uint64_t z = seed;
+    for (int64_t i = 0; i < count; ++i) {
+        z += 0x9E3779B97F4A7C15ull;
+        uint64_t t = z;
+        t = (t ^ (t >> 30)) * 0xBF58476D1CE4E5B9ull;
+        t = (t ^ (t >> 27)) * 0x94D049BB133111EBull;
+        t ^= t >> 31;
+        check((uint32_t)t);
+        check((uint32_t)(t >> 32));
+    }
+    // one block through block_dot with x = one-hot: each weight comes out alone
+    for (int pos = 0; pos < 32; ++pos) {
+        uint32_t words[4];
+        for (int w = 0; w < 4; ++w) words[w] = 0x9C2E4A71u * (uint32_t)(w + 3 + pos);
+        const uint4 q = make_uint4(words[0], words[1], words[2], words[3]);
+        float4 x[8];
+        for (int i = 0; i < 8; ++i) x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        float* xf = reinterpret_cast<float*>(x);
+        xf[pos] = 1.0f;
+        const float2 r = q4dev::block_dot(q, x);
+        const int byte = (pos % 16), hi = pos >= 16;
+        const uint32_t bv = (words[byte / 4] >> (8 * (byte % 4))) & 0xFFu;
+        const float want = (float)((int)(hi ? (bv >> 4) : (bv & 0xFu)) - 8);
+        bad += (r.x + r.y) != want;
+    }
+    return bad;
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// Device helpers for the sm_100a Q4_0 kernels: shared-memory barriers, bulk
+// (TMA engine) copies, programmatic dependent launch, bounded waits and the
+// register-resident nibble unpack of the decode mat-vec.
+#pragma once
+
+#include <cstdint>
+#include <cstring>
+#include <cmath>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace q4dev {
+
+// Time limit of every wait on an mbarrier (nanoseconds of %globaltimer). A wait
+// that gives up records Q4_ERR_TIMEOUT in the workspace header and the kernel
+// skips its math; copies of a few tens of KB normally land in microseconds.
+constexpr uint64_t kWaitLimitNs = 20ull * 1000 * 1000;
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make a freshly initialised barrier visible to the async (TMA) proxy.
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Returns true once the barrier's phase with the given parity has completed,
+// false if it did not within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_addr(bar);
+    const uint64_t start = global_ns();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (global_ns() - start > kWaitLimitNs) return false;
+    }
+}
+
+// Global -> shared bulk copy through the TMA engine, completing on `bar`.
+// dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel of the stream be scheduled,
+// and wait for the previous kernel's completion and memory flush.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__host__ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// Pairwise binary32 add / fused multiply-add: one packed f32x2 instruction on
+// sm_100a, two scalar operations when the same code runs on the host.
+__host__ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
+#ifdef __CUDA_ARCH__
+    return __fadd2_rn(a, b);
+#else
+    return f2(a.x + b.x, a.y + b.y);
+#endif
+}
+
+__host__ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+#ifdef __CUDA_ARCH__
+    return __ffma2_rn(a, b, c);
+#else
+    return f2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#endif
+}
+
+__host__ __device__ __forceinline__ float bits_f32(uint32_t u) {
+#ifdef __CUDA_ARCH__
+    return __uint_as_float(u);
+#else
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+#endif
+}
+
+// The four weight pairs of one 32-bit word of codes, as exact binary32 (q - 8).
+//
+// A word holds bytes 4w..4w+3 of a block. Byte 4w+m carries weight 4w+m in its
+// low nibble and weight 16+4w+m in its high nibble. A nibble at bit p of a
+// binary32 significand (p <= 19, so that it stays clear of the exponent field at
+// bits 23..30) becomes the value 2^(23-p) + q when OR-ed into the bit pattern of
+// 2^(23-p): its bits land exactly on the units place. Subtracting 2^(23-p) + 8
+// then gives q - 8 exactly. The nibbles at bits 20, 24 and 28 are read from the
+// word shifted right by 12, where they sit at bits 8, 12 and 16.
+//   lo01 = weights (4w,     4w+1)     bits 0, 8
+//   lo23 = weights (4w+2,   4w+3)     bits 16, 24 (-> 12 after the shift)
+//   hi01 = weights (16+4w,  16+4w+1)  bits 4, 12
+//   hi23 = weights (16+4w+2, 16+4w+3) bits 20, 28 (-> 8, 16 after the shift)
+struct Pairs {
+    float2 lo01, lo23, hi01, hi23;
+};
+
+__host__ __device__ __forceinline__ Pairs unpack_word(uint32_t q) {
+    const uint32_t s = q >> 12;
+    Pairs p;
+    p.lo01 = add2(f2(bits_f32((q & 0x0000000Fu) | 0x4B000000u),   // 2^23 + q
+                     bits_f32((q & 0x00000F00u) | 0x47000000u)),  // 2^15 + q
+                  f2(-8388616.0f, -32776.0f));
+    p.lo23 = add2(f2(bits_f32((q & 0x000F0000u) | 0x43000000u),   // 2^7 + q
+                     bits_f32((s & 0x0000F000u) | 0x45000000u)),  // 2^11 + q
+                  f2(-136.0f, -2056.0f));
+    p.hi01 = add2(f2(bits_f32((q & 0x000000F0u) | 0x49000000u),   // 2^19 + q
+                     bits_f32((q & 0x0000F000u) | 0x45000000u)),  // 2^11 + q
+                  f2(-524296.0f, -2056.0f));
+    p.hi23 = add2(f2(bits_f32((s & 0x00000F00u) | 0x47000000u),   // 2^15 + q
+                     bits_f32((s & 0x000F0000u) | 0x43000000u)),  // 2^7 + q
+                  f2(-32776.0f, -136.0f));
+    return p;
+}
+
+// Sum over one block of (q - 8) * x, with x given as 8 float4 chunks: chunk i
+// holds x[4i .. 4i+3] of the block. Returns two partial sums.
+__host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4 (&x)[8]) {
+    float2 acc = f2(0.0f, 0.0f);
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const Pairs p = unpack_word(words[w]);
+        acc = fma2(p.lo01, f2(x[w].x, x[w].y), acc);
+        acc = fma2(p.lo23, f2(x[w].z, x[w].w), acc);
+        acc = fma2(p.hi01, f2(x[w + 4].x, x[w + 4].y), acc);
+        acc = fma2(p.hi23, f2(x[w + 4].z, x[w + 4].w), acc);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+}  // namespace q4dev

@@ -1,0 +1,122 @@
+"""The C-ABI library on the CPU: it loads, exports what include/*.h declares,
+rejects bad arguments before touching CUDA, and its launch plans replay cleanly."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from quantized_decode_q4_b200 import q4, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(q4_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "q4_gemv" in names and "q4_layer_stack" in names and len(names) >= 20
+    lib = ctypes.CDLL(q4.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    assert q4.status_string(0) == "ok"
+    assert "misaligned" in q4.status_string(2)
+    assert q4.status_string(99) == "unknown status"
+
+
+def test_argument_errors_before_cuda():
+    L = q4.lib()
+    m = q4.q4_matrix(16, 16, 4, 33)  # k not a multiple of 32
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 256, 1 << 20, None) == 1
+    m = q4.q4_matrix(16, 16, 0, 64)  # n < 1
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 256, 1 << 20, None) == 1
+    m = q4.q4_matrix(24, 16, 4, 64)  # qs not 16-byte aligned
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 256, 1 << 20, None) == 2
+    m = q4.q4_matrix(16, 16, 4, 64)
+    assert L.q4_gemv(ctypes.byref(m), 20, 16, 256, 1 << 20, None) == 2   # x misaligned
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 0, 1 << 20, None) == 3     # no workspace
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 256, 8, None) == 3         # too small
+    assert L.q4_gemv(ctypes.byref(m), 16, 16, 272, 1 << 20, None) == 2   # ws alignment
+    assert L.q4_gemv_batched(ctypes.byref(m), 16, 0, 16, 256, 1 << 20, None) == 4
+    assert L.q4_gemv_batched(ctypes.byref(m), 16, 17, 16, 256, 1 << 20, None) == 4
+    assert L.q4_gemv(None, 16, 16, 256, 1 << 20, None) == 1
+    assert L.q4_pack(16, ctypes.byref(q4.q4_matrix(16, 16, 4, 40)), None) == 1
+    assert L.q4_dequant(ctypes.byref(m), 8, None) == 2
+
+
+def test_stack_group_rules():
+    L = q4.lib()
+    mats = (q4.q4_matrix * 3)(*[q4.q4_matrix(256, 256, 64, 64)] * 3)
+    xs = (ctypes.c_void_p * 3)(512, 512, 512)
+    ys = (ctypes.c_void_p * 3)(1024, 1024, 1024)
+    bad = (ctypes.c_int * 3)(0, 2, 1)   # groups must not decrease
+    s = q4.q4_stack(3, mats, xs, ys, bad)
+    assert L.q4_layer_stack(ctypes.byref(s), 1, 256, 1 << 20, None) == 1
+    assert L.q4_stack_workspace_bytes(ctypes.byref(s), 1) == 0
+    ok = (ctypes.c_int * 3)(0, 0, 1)
+    s = q4.q4_stack(3, mats, xs, ys, ok)
+    assert L.q4_stack_workspace_bytes(ctypes.byref(s), 1) >= 256
+    nine = (q4.q4_matrix * 9)(*[q4.q4_matrix(256, 256, 64, 64)] * 9)
+    x9 = (ctypes.c_void_p * 9)(*[512] * 9)
+    g9 = (ctypes.c_int * 9)(*[0] * 9)   # more than 8 GEMVs in a group
+    s = q4.q4_stack(9, nine, x9, x9, g9)
+    assert L.q4_stack_workspace_bytes(ctypes.byref(s), 1) == 0
+
+
+def _all_shapes():
+    shapes = set()
+    for wl in synth.workloads().values():
+        for g in wl.gemvs:
+            shapes.add((g.n, g.k))
+    return sorted(shapes)
+
+
+EDGE_SHAPES = [(1, 32), (17, 32), (1, 96), (5, 64), (33, 4128), (3, 28672), (50257, 768),
+               (16, 4096), (15, 4096), (2, 131072)]
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_launch_plans_replay_on_host(b):
+    for s in _all_shapes() + EDGE_SHAPES:
+        assert q4.check_plan([s], b) == 0, (s, b)
+    for wl in synth.workloads().values():
+        groups = {}
+        for g in wl.gemvs:
+            groups.setdefault(g.group, []).append((g.n, g.k))
+        for shapes in {tuple(v) for v in groups.values()}:
+            assert q4.check_plan(list(shapes), b) == 0, (shapes, b)
+
+
+def test_plan_properties():
+    info = q4.plan_info([(14336, 4096), (14336, 4096)], 1)
+    assert info["splits"] == [1, 1] and info["units"] == 1792 and info["ws_bytes"] == 256
+    assert info["smem"] <= 227 * 1024 // 4   # four CTAs fit on an SM
+    down = q4.plan_info([(4096, 14336)], 1)
+    assert down["splits"][0] >= 4            # K = 14336 does not fit one split
+
+
+def test_register_unpack_on_host():
+    assert q4.check_unpack(12345, 500000) == 0
+
+
+def test_interchange_matches_oracle():
+    rng = np.random.default_rng(5)
+    n, k = 7, 96
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    blocks = oracle.q4_pack(w)
+    qs_o, d_o = oracle.blocks_to_planes(blocks, n, k)
+    qs, d = q4.blocks_to_planes(blocks, n, k)
+    assert np.array_equal(qs, qs_o) and np.array_equal(d, d_o)
+    assert np.array_equal(q4.planes_to_blocks(qs, d, n, k), blocks)
