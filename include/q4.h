@@ -87,7 +87,7 @@ q4_status q4_plane_bytes(int64_t n, int64_t k, size_t* qs_bytes, size_t* d_bytes
  *   w   : device, binary32 [out->n][out->k], row-major, 16-byte aligned.
  *   out : out->qs, out->d, out->n, out->k filled in by the caller (planes
  *         allocated with q4_plane_bytes). Weights must be finite, with |w| small
- *         enough that d fits binary16 (|w| <= 524256); other inputs give
+ *         enough that d fits binary16 (|w| < 524160); other inputs give
  *         unspecified codes.
  * Errors: Q4_ERR_INVALID_ARG, Q4_ERR_MISALIGNED, Q4_ERR_CUDA. */
 q4_status q4_pack(const float* w, const q4_matrix* out, void* stream);
@@ -132,10 +132,8 @@ q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t
                   void* stream);
 
 /* q4_gemv_batched — Y[t] = W X[t] for t < b, 1 <= b <= 16 ("batch 1 to a few
- * tokens"). Each unpacked block is reused for every token; from b = 8 up the
- * product runs on the tensor cores with the codes dequantised to bf16 tiles in
- * shared memory ("Llamas on the Web" section 3, mat-mat path) and x split into
- * two bf16 parts so that the result keeps binary32 accuracy.
+ * tokens"). Each unpacked code word is reused for every token of a launch (up to
+ * 4 tokens per launch; larger b runs as several launches on the stream).
  *   X : device, binary32 [b][m->k] row-major, 16-byte aligned.
  *   Y : device, binary32 [b][m->n] row-major, 16-byte aligned.
  *   ws: as for q4_gemv with q4_workspace_bytes(n, k, b).
@@ -192,6 +190,11 @@ q4_status q4_planes_to_blocks(const uint8_t* qs, const uint16_t* d, int64_t n, i
 
 /* A static, human-readable name for a status code. */
 const char* q4_status_string(q4_status s);
+
+/* The CUDA runtime's message for the last CUDA call of this library that failed
+ * on the calling thread (what a Q4_ERR_CUDA status came from); "no error" if
+ * none has. The string is static. */
+const char* q4_last_cuda_error(void);
 
 /* Number of kernels this library has launched in this process (a diagnostic
  * counter; graph replays count the kernels they contain). */

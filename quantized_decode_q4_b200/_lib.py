@@ -75,6 +75,7 @@ def lib():
             "q4_planes_to_blocks": ([vp, vp, i64, i64, vp], c.c_int),
             "q4_status_string": ([c.c_int], c.c_char_p),
             "q4_launch_count": ([], c.c_uint64),
+            "q4_last_cuda_error": ([], c.c_char_p),
             "q4_debug_check_plan": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int], c.c_int),
             "q4_debug_plan_info": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int,
                                     c.POINTER(i64)], c.c_int),
@@ -90,6 +91,8 @@ def lib():
 
 def _check(status: int, where: str):
     if status != 0:
+        if status == 5:
+            where = f"{where} [{lib().q4_last_cuda_error().decode()}]"
         raise Q4Error(status, where)
 
 

@@ -22,7 +22,7 @@ cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblock
                         cudaStream_t stream);
 cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int64_t nblocks,
                            cudaStream_t stream);
-cudaError_t setup_gemv_kernels();
+cudaError_t setup_gemv_kernels(int optin_smem);
 cudaError_t launch_gemv(const q4plan::GemvParams& P, bool pdl, cudaStream_t stream);
 }  // namespace q4k
 
@@ -32,11 +32,19 @@ using q4plan::GemvParams;
 namespace {
 
 std::atomic<uint64_t> g_launches{0};
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Record a failed CUDA call for q4_last_cuda_error() and map it to Q4_ERR_CUDA.
+bool cuda_failed(cudaError_t e) {
+    if (e == cudaSuccess) return false;
+    g_last_cuda_error = e;
+    return true;
+}
 
 // CTAs a launch aims for before K is split further: two per SM of a B200.
 constexpr int64_t kTargetUnits = 2 * 148;
 constexpr int kMaxCudaCoreBatch = 4;
-constexpr uint32_t kMaxSmem = 227 * 1024;
+constexpr uint32_t kMaxSmem = 226 * 1024;  // below the opt-in limit minus static smem
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -62,8 +70,15 @@ struct Shape {
 };
 
 // Plan one launch over `count` GEMVs of the given shapes. Fills everything in P
-// except the pointers, and the workspace bytes it needs.
-q4_status plan_shapes(const Shape* sh, int count, int batch, GemvParams* P, size_t* ws_bytes) {
+// except the pointers. Workspace layout of a call: [256-byte status header]
+// [split-K tickets, one uint32 per row tile of every split GEMV][partial sums].
+// Tickets start right after the header; partial sums start at `part_base` bytes,
+// which a stack sets past the largest ticket region of all its groups so that no
+// partial sum of any group overlaps any ticket. Every call zeroes its ticket
+// region before its first kernel. Returns the tickets used (*tickets) and the
+// end of the partial sums (*ws_end, bytes).
+q4_status plan_shapes(const Shape* sh, int count, int batch, int64_t part_base, GemvParams* P,
+                      int64_t* tickets, int64_t* ws_end) {
     if (count < 1 || count > Q4_MAX_GROUP || batch < 1 || batch > kMaxCudaCoreBatch)
         return Q4_ERR_INVALID_ARG;
     std::memset(P, 0, sizeof *P);
@@ -76,7 +91,8 @@ q4_status plan_shapes(const Shape* sh, int count, int batch, GemvParams* P, size
     }
     const int64_t factor = base_units >= kTargetUnits ? 1 : ceil_div(kTargetUnits, base_units);
     int64_t units = 0;
-    int64_t off = q4plan::kHeaderBytes;
+    int64_t tick = 0;
+    int64_t part = part_base;
     int nbs_max = 1;
     for (int i = 0; i < count; ++i) {
         GemvDesc& G = P->g[i];
@@ -95,15 +111,16 @@ q4_status plan_shapes(const Shape* sh, int count, int batch, GemvParams* P, size
         G.row_tiles = (int32_t)tiles;
         G.unit_begin = (int32_t)units;
         if (S > 1) {
-            G.ticket_off = off / 4;
-            off += round_up(tiles * 4, 256);
-            G.part_off = off / 4;
-            off += round_up((int64_t)batch * S * sh[i].n * 4, 256);
+            G.ticket_off = q4plan::kHeaderBytes / 4 + tick;
+            tick += tiles;
+            G.part_off = part / 4;
+            part += round_up((int64_t)batch * S * sh[i].n * 4, 256);
         }
         units += tiles * S;
         nbs_max = std::max<int>(nbs_max, (int)nbs);
         if (units > INT_MAX / 2) return Q4_ERR_INVALID_ARG;
     }
+    if (q4plan::kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
     P->count = count;
     P->total_units = (int32_t)units;
     P->batch = batch;
@@ -117,8 +134,20 @@ q4_status plan_shapes(const Shape* sh, int count, int batch, GemvParams* P, size
     P->smem_total = q4plan::kBarrierBytes + P->smem_x +
                     q4plan::kWarps * (P->smem_qs_warp + P->smem_d_warp);
     if (P->smem_total > kMaxSmem) return Q4_ERR_UNSUPPORTED;
-    *ws_bytes = (size_t)off;
+    *tickets = tick;
+    *ws_end = part;
     return Q4_OK;
+}
+
+// Tickets of one launch, found by planning with room for any ticket count.
+q4_status count_tickets(const Shape* sh, int count, int batch, int64_t* tickets) {
+    GemvParams P;
+    int64_t end = 0;
+    return plan_shapes(sh, count, batch, INT64_MAX / 4, &P, tickets, &end);
+}
+
+int64_t part_base_for(int64_t tickets) {
+    return q4plan::kHeaderBytes + round_up(4 * tickets, 256);
 }
 
 // Token chunks: batches above the CUDA-core kernel's width run as several
@@ -130,16 +159,17 @@ bool g_dev_ready[64];
 
 q4_status ensure_device() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return Q4_ERR_CUDA;
+    if (cuda_failed(cudaGetDevice(&dev))) return Q4_ERR_CUDA;
     if (dev < 0 || dev >= 64) return Q4_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_dev_mu);
     if (g_dev_ready[dev]) return Q4_OK;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    int major = 0, minor = 0, optin = 0;
+    if (cuda_failed(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) ||
+        cuda_failed(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) ||
+        cuda_failed(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)))
         return Q4_ERR_CUDA;
     if (major != 10 || minor != 0) return Q4_ERR_UNSUPPORTED;
-    if (q4k::setup_gemv_kernels() != cudaSuccess) return Q4_ERR_CUDA;
+    if (cuda_failed(q4k::setup_gemv_kernels(optin))) return Q4_ERR_CUDA;
     g_dev_ready[dev] = true;
     return Q4_OK;
 }
@@ -150,8 +180,10 @@ struct GemvCall {
     float* y;
 };
 
-// Validate and plan one group for `b` tokens; returns the workspace bytes needed.
-q4_status check_group(const GemvCall* calls, int count, int b, size_t* ws_need) {
+// Validate one group for `b` tokens; returns its largest ticket count over the
+// token chunks and the partial-sum bytes it needs past the ticket region.
+q4_status check_group(const GemvCall* calls, int count, int b, int64_t* tickets,
+                      int64_t* part_bytes) {
     if (count < 1 || count > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
     if (b < 1 || b > Q4_MAX_BATCH) return Q4_ERR_UNSUPPORTED;
     Shape sh[Q4_MAX_GROUP];
@@ -162,15 +194,17 @@ q4_status check_group(const GemvCall* calls, int count, int b, size_t* ws_need) 
         if (!aligned(calls[i].x, 16) || !aligned(calls[i].y, 16)) return Q4_ERR_MISALIGNED;
         sh[i] = {calls[i].m.n, calls[i].m.k};
     }
-    size_t need = 0;
+    int64_t tmax = 0, pmax = 0;
     for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
         GemvParams P;
-        size_t w = 0;
-        q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), &P, &w);
+        int64_t t = 0, end = 0;
+        q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), 0x40000000LL, &P, &t, &end);
         if (s != Q4_OK) return s;
-        need = std::max(need, w);
+        tmax = std::max(tmax, t);
+        pmax = std::max(pmax, end - (int64_t)0x40000000LL);
     }
-    *ws_need = need;
+    *tickets = tmax;
+    *part_bytes = pmax;
     return Q4_OK;
 }
 
@@ -180,18 +214,18 @@ q4_status check_ws(void* ws, size_t ws_bytes, size_t need) {
     return Q4_OK;
 }
 
-// Enqueue one group (all token chunks). The first launch may use PDL only if
-// `pdl_first` is set.
-q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, bool pdl_first,
-                       cudaStream_t stream) {
+// Enqueue one group (all token chunks) with partial sums from `part_base`. The
+// first launch may use PDL only if `pdl_first` is set.
+q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_t part_base,
+                       bool pdl_first, cudaStream_t stream) {
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {calls[i].m.n, calls[i].m.k};
     bool pdl = pdl_first;
     for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
         const int bt = chunk_tokens(b, c0);
         GemvParams P;
-        size_t w = 0;
-        q4_status s = plan_shapes(sh, count, bt, &P, &w);
+        int64_t t = 0, end = 0;
+        q4_status s = plan_shapes(sh, count, bt, part_base, &P, &t, &end);
         if (s != Q4_OK) return s;
         for (int i = 0; i < count; ++i) {
             P.g[i].qs = calls[i].m.qs;
@@ -200,10 +234,19 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, bool p
             P.g[i].y = calls[i].y + (int64_t)c0 * calls[i].m.n;
         }
         P.ws = static_cast<uint32_t*>(ws);
-        if (q4k::launch_gemv(P, pdl, stream) != cudaSuccess) return Q4_ERR_CUDA;
+        if (cuda_failed(q4k::launch_gemv(P, pdl, stream))) return Q4_ERR_CUDA;
         g_launches.fetch_add(1, std::memory_order_relaxed);
         pdl = true;
     }
+    return Q4_OK;
+}
+
+// Zero the ticket region of a call before its first kernel.
+q4_status clear_tickets(void* ws, int64_t tickets, cudaStream_t stream) {
+    if (tickets == 0) return Q4_OK;
+    if (cuda_failed(cudaMemsetAsync(static_cast<uint8_t*>(ws) + q4plan::kHeaderBytes, 0,
+                                    (size_t)(4 * tickets), stream)))
+        return Q4_ERR_CUDA;
     return Q4_OK;
 }
 
@@ -223,21 +266,25 @@ q4_status stack_groups(const q4_stack* s, std::vector<std::pair<int, int>>* out)
     return Q4_OK;
 }
 
+// Validate a stack; returns the ticket region shared by all groups and the
+// workspace bytes needed.
 q4_status stack_check(const q4_stack* s, int b, std::vector<std::pair<int, int>>* groups,
-                      size_t* need) {
+                      int64_t* tickets, size_t* need) {
     q4_status st = stack_groups(s, groups);
     if (st != Q4_OK) return st;
-    size_t mx = 0;
+    int64_t tmax = 0, pmax = 0;
     for (auto& g : *groups) {
         GemvCall calls[Q4_MAX_GROUP];
         for (int i = g.first; i < g.second; ++i)
             calls[i - g.first] = {s->mats[i], s->x[i], s->y[i]};
-        size_t w = 0;
-        st = check_group(calls, g.second - g.first, b, &w);
+        int64_t t = 0, p = 0;
+        st = check_group(calls, g.second - g.first, b, &t, &p);
         if (st != Q4_OK) return st;
-        mx = std::max(mx, w);
+        tmax = std::max(tmax, t);
+        pmax = std::max(pmax, p);
     }
-    *need = mx;
+    *tickets = tmax;
+    *need = (size_t)(part_base_for(tmax) + pmax);
     return Q4_OK;
 }
 
@@ -292,21 +339,23 @@ q4_status q4_dequant(const q4_matrix* m, float* w_out, void* stream) {
 
 size_t q4_workspace_bytes(int64_t n, int64_t k, int b) {
     if (check_shape(n, k) != Q4_OK || b < 1 || b > Q4_MAX_BATCH) return 0;
-    size_t need = 0;
     const Shape sh = {n, k};
+    int64_t tmax = 0, pmax = 0;
     for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
         GemvParams P;
-        size_t w = 0;
-        if (plan_shapes(&sh, 1, chunk_tokens(b, c0), &P, &w) != Q4_OK) return 0;
-        need = std::max(need, w);
+        int64_t t = 0, end = 0;
+        if (plan_shapes(&sh, 1, chunk_tokens(b, c0), 0x40000000LL, &P, &t, &end) != Q4_OK)
+            return 0;
+        tmax = std::max(tmax, t);
+        pmax = std::max(pmax, end - (int64_t)0x40000000LL);
     }
-    return need;
+    return (size_t)(part_base_for(tmax) + pmax);
 }
 
 q4_status q4_workspace_init(void* ws, size_t ws_bytes, void* stream) {
     if (!ws || ws_bytes < (size_t)q4plan::kHeaderBytes) return Q4_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return Q4_ERR_MISALIGNED;
-    if (cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cuda_failed(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream))))
         return Q4_ERR_CUDA;
     return Q4_OK;
 }
@@ -315,9 +364,9 @@ q4_status q4_workspace_status(const void* ws, void* stream) {
     if (!ws) return Q4_ERR_WORKSPACE;
     uint32_t flag = 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(&flag, ws, sizeof flag, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    if (cuda_failed(cudaMemcpyAsync(&flag, ws, sizeof flag, cudaMemcpyDeviceToHost, st)))
         return Q4_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return Q4_ERR_CUDA;
+    if (cuda_failed(cudaStreamSynchronize(st))) return Q4_ERR_CUDA;
     return flag ? Q4_ERR_TIMEOUT : Q4_OK;
 }
 
@@ -325,12 +374,15 @@ q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, v
                           size_t ws_bytes, void* stream) {
     if (!m) return Q4_ERR_INVALID_ARG;
     GemvCall call = {*m, X, Y};
-    size_t need = 0;
-    q4_status s = check_group(&call, 1, b, &need);
+    int64_t tickets = 0, part = 0;
+    q4_status s = check_group(&call, 1, b, &tickets, &part);
     if (s != Q4_OK) return s;
-    if ((s = check_ws(ws, ws_bytes, need)) != Q4_OK) return s;
+    const int64_t base = part_base_for(tickets);
+    if ((s = check_ws(ws, ws_bytes, (size_t)(base + part))) != Q4_OK) return s;
     if ((s = ensure_device()) != Q4_OK) return s;
-    return launch_group(&call, 1, b, ws, false, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_tickets(ws, tickets, st)) != Q4_OK) return s;
+    return launch_group(&call, 1, b, ws, base, false, st);
 }
 
 q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t ws_bytes,
@@ -340,25 +392,29 @@ q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t
 
 size_t q4_stack_workspace_bytes(const q4_stack* s, int b) {
     std::vector<std::pair<int, int>> groups;
+    int64_t tickets = 0;
     size_t need = 0;
-    if (stack_check(s, b, &groups, &need) != Q4_OK) return 0;
+    if (stack_check(s, b, &groups, &tickets, &need) != Q4_OK) return 0;
     return need;
 }
 
 q4_status q4_layer_stack(const q4_stack* s, int b, void* ws, size_t ws_bytes, void* stream) {
     std::vector<std::pair<int, int>> groups;
+    int64_t tickets = 0;
     size_t need = 0;
-    q4_status st = stack_check(s, b, &groups, &need);
+    q4_status st = stack_check(s, b, &groups, &tickets, &need);
     if (st != Q4_OK) return st;
     if ((st = check_ws(ws, ws_bytes, need)) != Q4_OK) return st;
     if ((st = ensure_device()) != Q4_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = clear_tickets(ws, tickets, cs)) != Q4_OK) return st;
+    const int64_t base = part_base_for(tickets);
     bool first = true;
     for (auto& g : groups) {
         GemvCall calls[Q4_MAX_GROUP];
         for (int i = g.first; i < g.second; ++i)
             calls[i - g.first] = {s->mats[i], s->x[i], s->y[i]};
-        st = launch_group(calls, g.second - g.first, b, ws, !first,
-                          static_cast<cudaStream_t>(stream));
+        st = launch_group(calls, g.second - g.first, b, ws, base, !first, cs);
         if (st != Q4_OK) return st;
         first = false;
     }
@@ -370,28 +426,30 @@ q4_status q4_stack_graph_create(const q4_stack* s, int b, void* ws, size_t ws_by
     if (!out || !stream) return Q4_ERR_INVALID_ARG;
     *out = nullptr;
     std::vector<std::pair<int, int>> groups;
+    int64_t tickets = 0;
     size_t need = 0;
-    q4_status st = stack_check(s, b, &groups, &need);
+    q4_status st = stack_check(s, b, &groups, &tickets, &need);
     if (st != Q4_OK) return st;
     if ((st = check_ws(ws, ws_bytes, need)) != Q4_OK) return st;
     if ((st = ensure_device()) != Q4_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(cs, &cap) != cudaSuccess) return Q4_ERR_CUDA;
+    if (cuda_failed(cudaStreamIsCapturing(cs, &cap))) return Q4_ERR_CUDA;
     if (cap != cudaStreamCaptureStatusNone) return Q4_ERR_INVALID_ARG;
-    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    if (cuda_failed(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)))
         return Q4_ERR_CUDA;
     const uint64_t before = g_launches.load();
     q4_status run = q4_layer_stack(s, b, ws, ws_bytes, stream);
     g_launches.store(before);  // captured launches do not run now
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(cs, &graph);
+    cuda_failed(e);
     if (run != Q4_OK || e != cudaSuccess) {
         if (graph) cudaGraphDestroy(graph);
         return run != Q4_OK ? run : Q4_ERR_CUDA;
     }
     cudaGraphExec_t exec = nullptr;
-    if (cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+    if (cuda_failed(cudaGraphInstantiate(&exec, graph, 0))) {
         cudaGraphDestroy(graph);
         return Q4_ERR_CUDA;
     }
@@ -410,7 +468,7 @@ q4_status q4_stack_graph_create(const q4_stack* s, int b, void* ws, size_t ws_by
 
 q4_status q4_graph_launch(q4_graph g, void* stream) {
     if (!g) return Q4_ERR_INVALID_ARG;
-    if (cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cuda_failed(cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream))))
         return Q4_ERR_CUDA;
     g_launches.fetch_add(g->kernels, std::memory_order_relaxed);
     return Q4_OK;
@@ -464,6 +522,8 @@ const char* q4_status_string(q4_status s) {
 
 uint64_t q4_launch_count(void) { return g_launches.load(); }
 
+const char* q4_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
 // ---------------------------------------------------------------------------
 // host-side diagnostics
 // ---------------------------------------------------------------------------
@@ -473,13 +533,15 @@ q4_status q4_debug_plan_info(const int64_t* n, const int64_t* k, int count, int 
         return Q4_ERR_INVALID_ARG;
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
+    int64_t tickets = 0, end = 0;
+    q4_status s = count_tickets(sh, count, b, &tickets);
+    if (s != Q4_OK) return s;
     GemvParams P;
-    size_t w = 0;
-    q4_status s = plan_shapes(sh, count, b, &P, &w);
+    s = plan_shapes(sh, count, b, part_base_for(tickets), &P, &tickets, &end);
     if (s != Q4_OK) return s;
     out[0] = P.total_units;
     out[1] = P.smem_total;
-    out[2] = (int64_t)w;
+    out[2] = end;
     for (int i = 0; i < count; ++i) out[3 + i] = P.g[i].splits;
     return Q4_OK;
 }
@@ -490,8 +552,11 @@ int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b) {
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
     GemvParams P;
-    size_t ws_bytes = 0;
-    if (plan_shapes(sh, count, b, &P, &ws_bytes) != Q4_OK) return 2;
+    int64_t tickets = 0, end = 0;
+    if (count_tickets(sh, count, b, &tickets) != Q4_OK) return 2;
+    const int64_t base = part_base_for(tickets);
+    if (plan_shapes(sh, count, b, base, &P, &tickets, &end) != Q4_OK) return 2;
+    const size_t ws_bytes = (size_t)end;
     if (P.smem_total > kMaxSmem) return 3;
     if (P.smem_x % 16 || P.smem_qs_warp % 16 || P.smem_d_warp % 16) return 4;
     if ((int64_t)kBarrierBytes < (int64_t)kWarps * 8) return 5;
@@ -552,21 +617,24 @@ int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b) {
         if (G.splits > 1) {
             if ((G.ticket_off + G.row_tiles) * 4 > (int64_t)ws_bytes) return 28;
             if ((G.part_off + (int64_t)b * G.splits * G.n) * 4 > (int64_t)ws_bytes) return 29;
-            if (G.ticket_off * 4 < kHeaderBytes || G.part_off * 4 < kHeaderBytes) return 30;
+            if (G.ticket_off * 4 < kHeaderBytes || G.part_off * 4 < base) return 30;
+            if ((G.ticket_off + G.row_tiles) * 4 > base) return 34;  // tickets before partials
         }
         ++units_seen;
     }
     for (int i = 0; i < count; ++i)
         for (uint8_t c : cover[i])
             if (!c) return 31;
-    // workspace regions of different GEMVs do not overlap
+    // ticket ranges of different GEMVs are disjoint, and so are partial-sum ranges
     for (int i = 0; i < count; ++i)
         for (int j = i + 1; j < count; ++j) {
             const GemvDesc &A = P.g[i], &B = P.g[j];
             if (A.splits < 2 || B.splits < 2) continue;
-            const int64_t a0 = A.ticket_off * 4, a1 = (A.part_off + (int64_t)b * A.splits * A.n) * 4;
-            const int64_t b0 = B.ticket_off * 4, b1 = (B.part_off + (int64_t)b * B.splits * B.n) * 4;
-            if (a0 < b1 && b0 < a1) return 32;
+            if (A.ticket_off < B.ticket_off + B.row_tiles && B.ticket_off < A.ticket_off + A.row_tiles)
+                return 32;
+            const int64_t a1 = A.part_off + (int64_t)b * A.splits * A.n;
+            const int64_t b1 = B.part_off + (int64_t)b * B.splits * B.n;
+            if (A.part_off < b1 && B.part_off < a1) return 35;
         }
     return units_seen == P.total_units ? 0 : 33;
 }

@@ -254,17 +254,23 @@ __global__ void __launch_bounds__(kThreads) gemv_bs_kernel(const __grid_constant
     if (G.splits > 1) finish_splits(P, G, u.tile, B);
 }
 
-cudaError_t setup_gemv_kernels() {
-    const int max_smem = 227 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(gemv_b1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         max_smem);
+// Allow each GEMV kernel the device's opt-in shared memory minus its static
+// shared memory (the per-block limit covers both).
+template <typename K>
+static cudaError_t allow_dynamic_smem(K kernel, int optin) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemv_bs_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemv_bs_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(gemv_bs_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                max_smem);
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - (int)fa.sharedSizeBytes);
+}
+
+cudaError_t setup_gemv_kernels(int optin_smem) {
+    cudaError_t e = allow_dynamic_smem(gemv_b1_kernel, optin_smem);
+    if (e == cudaSuccess) e = allow_dynamic_smem(gemv_bs_kernel<2>, optin_smem);
+    if (e == cudaSuccess) e = allow_dynamic_smem(gemv_bs_kernel<3>, optin_smem);
+    if (e == cudaSuccess) e = allow_dynamic_smem(gemv_bs_kernel<4>, optin_smem);
+    return e;
 }
 
 cudaError_t launch_gemv(const GemvParams& P, bool pdl, cudaStream_t stream) {

@@ -28,9 +28,10 @@ def assert_gemv_close(y_gpu, y_ref, abs_sum, what=""):
     y_gpu = np.asarray(y_gpu, dtype=np.float64)
     err = np.abs(y_gpu - y_ref)
     bound = REL_TOL * abs_sum + ABS_TOL
-    bad = np.nonzero(~(err <= bound))[0]
+    bad = np.flatnonzero(~(err <= bound))
     assert bad.size == 0, (f"{what}: {bad.size} of {y_ref.size} outputs outside tolerance; "
-                           f"first {bad[:5]}: gpu {y_gpu.ravel()[bad[:5]]} ref {y_ref.ravel()[bad[:5]]}")
+                           f"first flat indexes {bad[:5]}: gpu {y_gpu.ravel()[bad[:5]]} "
+                           f"ref {y_ref.ravel()[bad[:5]]}")
     return float(np.max(err / np.maximum(bound, 1e-300))) if err.size else 0.0
 
 

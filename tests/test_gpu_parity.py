@@ -189,3 +189,26 @@ def test_launch_counter_counts_kernels():
     q4.gemv(m, x)
     q4.gemv_batched(m, torch.randn(6, 256, device="cuda"))  # 4 + 2 tokens: two launches
     assert q4.launch_count() - c0 == 3
+
+
+def test_workspace_shared_by_different_shapes():
+    """Calls with different split-K layouts reuse one workspace in any order."""
+    shapes = [(1024, 4096), (128, 512), (4096, 14336), (1408, 512), (1024, 4096)]
+    need = max(q4.workspace_bytes(n, k, 4) for n, k in shapes)
+    ws = q4.workspace(need)
+    for i, (n, k) in enumerate(shapes):
+        w = host_matrix(13, i, n, k) if n * k <= FULL_CHECK_LIMIT else None
+        if w is None:
+            wg = synth.matrix(13, i, n, k, synth.WEIGHT_STD, device="cuda")
+            m = q4.pack(wg)
+            rows = sample_rows(n, 16, i)
+            w_rows = synth.matrix_rows(13, i, k, rows, synth.WEIGHT_STD).numpy()
+        else:
+            m = gpu_matrix_from_host(w)
+            rows = list(range(n))
+            w_rows = w
+        for b in (1, 3):
+            X = synth.normal(13, 500 + i, 0, b * k, 1.0).numpy().reshape(b, k)
+            Y = q4.gemv_batched(m, torch.from_numpy(X).cuda(), ws=ws).cpu().numpy()
+            Y_ref, S = oracle.q4_gemv_batched(oracle.q4_pack(w_rows), len(rows), k, X)
+            assert_gemv_close(Y[:, rows], Y_ref, S, f"{n}x{k} b={b} shared ws")
