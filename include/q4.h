@@ -141,6 +141,30 @@ q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t
 q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* q4_gemv_noalloc — q4_gemv without a caller workspace, for callers that cannot
+ * allocate device memory: a plugin inside a host application that owns every
+ * device allocation, a runtime whose memory budget is fixed after start-up, or a
+ * latency-critical path that must not call cudaMalloc because it can synchronise
+ * the whole device. The pages have no counterpart of this call.
+ * Same arguments, result and accuracy as q4_gemv, minus ws and ws_bytes; x and y
+ * are still the caller's device buffers. Split-K scratch (status header,
+ * tickets, partial sums) lives in one fixed device array of 1 MiB
+ * (1,048,576 bytes) inside the library, which every GPU that loads the library
+ * holds until the process exits. Nothing is allocated or
+ * freed by this call.
+ *   - A matrix whose scratch need, q4_workspace_bytes(n, k, 1), exceeds that size
+ *     is rejected with Q4_ERR_WORKSPACE before anything is enqueued (every matrix
+ *     of the 8B-class layer needs at most 66,816 bytes).
+ *   - The first call on each device looks up the array's device address and
+ *     configures the kernels for that device; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents; each call clears the tickets it uses before its kernel. Calls
+ *     that overlap on the GPU (for instance on two streams) race on the array:
+ *     serialise them.
+ * Errors: as q4_gemv. */
+q4_status q4_gemv_noalloc(const q4_matrix* m, const float* x, float* y, void* stream);
+
 /* A decode step: `count` GEMVs in dependency groups. group[i] is the group of
  * GEMV i; groups are non-decreasing and run in order; the GEMVs of one group
  * (at most Q4_MAX_GROUP) are independent and run in one launch. x[i] is device

@@ -507,6 +507,62 @@ q4_status q4_planes_to_blocks(const uint8_t* qs, const uint16_t* d, int64_t n, i
     return Q4_OK;
 }
 
+// ---------------------------------------------------------------------------
+// q4_gemv_noalloc: the batch-1 GEMV with its split-K scratch in a fixed device
+// array instead of a caller workspace.
+//
+// Some callers cannot hand the library a workspace: a plugin inside a host
+// application that owns every device allocation, a runtime with a fixed memory
+// budget that forbids allocating after start-up, or a latency-critical path that
+// must not call cudaMalloc because it can synchronise the whole device. For
+// them the scratch lives in the array below, which every GPU that loads this
+// library holds until the process exits.
+// ---------------------------------------------------------------------------
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB per GPU
+
+// Header, split-K tickets and partial sums of q4_gemv_noalloc. In host code this
+// name is only a stand-in for the symbol, never a device address: the address
+// comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device (looked up on the
+// first call made while that device is current).
+q4_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cuda_failed(cudaGetDevice(&dev))) return Q4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return Q4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cuda_failed(cudaGetSymbolAddress(&p, g_noalloc_scratch))) return Q4_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return Q4_OK;
+}
+}  // namespace
+
+q4_status q4_gemv_noalloc(const q4_matrix* m, const float* x, float* y, void* stream) {
+    if (!m) return Q4_ERR_INVALID_ARG;
+    GemvCall call = {*m, x, y};
+    int64_t tickets = 0, part = 0;
+    q4_status s = check_group(&call, 1, 1, &tickets, &part);
+    if (s != Q4_OK) return s;
+    const int64_t base = part_base_for(tickets);
+    if ((size_t)(base + part) > kNoAllocScratchBytes) return Q4_ERR_WORKSPACE;
+    if ((s = ensure_device()) != Q4_OK) return s;
+    void* scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != Q4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_tickets(scratch, tickets, st)) != Q4_OK) return s;
+    return launch_group(&call, 1, 1, scratch, base, false, st);
+}
+
 const char* q4_status_string(q4_status s) {
     switch (s) {
         case Q4_OK: return "ok";
