@@ -154,7 +154,7 @@ q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, v
  * freed by this call.
  *   - A matrix whose scratch need, q4_workspace_bytes(n, k, 1), exceeds that size
  *     is rejected with Q4_ERR_WORKSPACE before anything is enqueued (every matrix
- *     of the 8B-class layer needs at most 66,816 bytes).
+ *     of the 8B-class layer needs at most 82,176 bytes).
  *   - The first call on each device looks up the array's device address and
  *     configures the kernels for that device; make that first call before any
  *     stream capture.

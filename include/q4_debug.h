@@ -25,6 +25,13 @@ extern "C" {
  * the number of the first failed check (see q4_api.cu). */
 int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b);
 
+/* The same replay for the persistent batch-1 streaming kernel: every CTA's unit
+ * range, every warp's chunk sequence (the copy issuer's and the consumer's must
+ * agree chunk for chunk), every bulk copy's source and stage slot, exactly-once
+ * coverage of every (row, block), and split-K tickets and partial sums inside
+ * their workspace regions. Returns 0 when every check holds. */
+int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count);
+
 /* Summary of the plan above: out[0] = CTAs (units), out[1] = dynamic shared
  * memory bytes per CTA, out[2] = workspace bytes, out[3 + i] = K splits of GEMV i.
  * Returns Q4_OK or Q4_ERR_INVALID_ARG. */
@@ -35,6 +42,16 @@ q4_status q4_debug_plan_info(const int64_t* n, const int64_t* k, int count, int 
  * nibble, comparing with plain nibble extraction. Returns the number of
  * mismatching values (0 when correct). */
 int64_t q4_debug_check_unpack(uint64_t seed, int64_t count);
+
+/* Check the batch-1 kernel's integer block dot product on the host (the same
+ * source compiled for the CPU): every |X| <= 8,355,711 splits into three digits
+ * in -128..127 that add back up, and for `blocks` pseudo-random blocks of codes
+ * and activations over many magnitudes (zeros, 1e-20, 1e30, one dominant
+ * element) the block sum times its scale is within
+ * sum_j |q_j - 8| (s/2 + |x_j| 2^-22) + 2^-22 |exact| of the exact sum; blocks
+ * with max|x| < 1e-30 (taken as zero) within sum_j |q_j - 8| |x_j|. Returns
+ * the number of failures (0 when correct). */
+int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks);
 
 #ifdef __cplusplus
 }

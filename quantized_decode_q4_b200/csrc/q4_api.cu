@@ -15,7 +15,9 @@
 #include "../../include/q4.h"
 #include "../../include/q4_debug.h"
 #include "q4_device.cuh"
+#include "q4_intdot.cuh"
 #include "q4_plan.h"
+#include "q4_stream_plan.h"
 
 namespace q4k {
 cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblocks,
@@ -24,6 +26,8 @@ cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int
                            cudaStream_t stream);
 cudaError_t setup_gemv_kernels(int optin_smem);
 cudaError_t launch_gemv(const q4plan::GemvParams& P, bool pdl, cudaStream_t stream);
+cudaError_t setup_stream_kernel(int optin_smem);
+cudaError_t launch_stream(const q4s::Params& P, int grid, bool pdl, cudaStream_t stream);
 }  // namespace q4k
 
 using q4plan::GemvDesc;
@@ -150,6 +154,57 @@ int64_t part_base_for(int64_t tickets) {
     return q4plan::kHeaderBytes + round_up(4 * tickets, 256);
 }
 
+// Streaming (batch 1) plan over `count` GEMVs: splits, units, grid, tickets and
+// partial sums laid out as for plan_shapes.
+constexpr int kNumSMs = 148;
+
+q4_status plan_stream(const Shape* sh, int count, int64_t part_base, q4s::Params* P, int* grid,
+                      int64_t* tickets, int64_t* ws_end) {
+    if (count < 1 || count > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
+    std::memset(P, 0, sizeof *P);
+    int64_t base_rows = 0;
+    for (int i = 0; i < count; ++i) {
+        q4_status s = check_shape(sh[i].n, sh[i].k);
+        if (s != Q4_OK) return s;
+        base_rows += sh[i].n * ceil_div(sh[i].k / Q4_QK, q4s::kMaxSplitBlocks);
+    }
+    // enough rows for one full tile per warp of the grid, splitting K (in whole
+    // sub-steps of 32 blocks) when the matrices are short
+    const int64_t target = (int64_t)kNumSMs * Q4_STREAM_CTAS_PER_SM * q4s::kWarps * q4s::kRows;
+    const int64_t factor = base_rows >= target ? 1 : ceil_div(target, base_rows);
+    int64_t rows = 0, tick = 0, part = part_base;
+    for (int i = 0; i < count; ++i) {
+        q4s::Desc& G = P->g[i];
+        const int64_t nb = sh[i].k / Q4_QK;
+        const int64_t smin = ceil_div(nb, q4s::kMaxSplitBlocks);
+        const int64_t smax = std::max<int64_t>(smin, nb / 32);
+        const int64_t S0 = std::min(smin * factor, smax);
+        int64_t nbs = ceil_div(nb, S0);
+        if (S0 > 1) nbs = std::min<int64_t>(round_up(nbs, 32), q4s::kMaxSplitBlocks);
+        const int64_t S = ceil_div(nb, nbs);
+        G.n = sh[i].n;
+        G.nb = (int32_t)nb;
+        G.splits = (int32_t)S;
+        G.nb_split = (int32_t)nbs;
+        G.row_begin = rows;
+        if (S > 1) {
+            G.ticket_off = q4plan::kHeaderBytes / 4 + tick;
+            tick += sh[i].n;
+            G.part_off = part / 4;
+            part += round_up(S * sh[i].n * 4, 256);
+        }
+        rows += sh[i].n * S;
+        if (rows >= (int64_t(1) << 31)) return Q4_ERR_INVALID_ARG;  // 32-bit row space
+    }
+    if (q4plan::kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
+    P->count = count;
+    P->total_rows = rows;
+    *grid = (int)std::min<int64_t>((int64_t)kNumSMs * Q4_STREAM_CTAS_PER_SM, rows);
+    *tickets = tick;
+    *ws_end = part;
+    return Q4_OK;
+}
+
 // Token chunks: batches above the CUDA-core kernel's width run as several
 // launches of at most kMaxCudaCoreBatch tokens.
 int chunk_tokens(int b, int c0) { return std::min(kMaxCudaCoreBatch, b - c0); }
@@ -170,6 +225,7 @@ q4_status ensure_device() {
         return Q4_ERR_CUDA;
     if (major != 10 || minor != 0) return Q4_ERR_UNSUPPORTED;
     if (cuda_failed(q4k::setup_gemv_kernels(optin))) return Q4_ERR_CUDA;
+    if (cuda_failed(q4k::setup_stream_kernel(optin))) return Q4_ERR_CUDA;
     g_dev_ready[dev] = true;
     return Q4_OK;
 }
@@ -195,7 +251,16 @@ q4_status check_group(const GemvCall* calls, int count, int b, int64_t* tickets,
         sh[i] = {calls[i].m.n, calls[i].m.k};
     }
     int64_t tmax = 0, pmax = 0;
-    for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
+    if (b == 1) {
+        q4s::Params P;
+        int grid = 0;
+        int64_t t = 0, end = 0;
+        q4_status s = plan_stream(sh, count, 0x40000000LL, &P, &grid, &t, &end);
+        if (s != Q4_OK) return s;
+        tmax = t;
+        pmax = end - (int64_t)0x40000000LL;
+    }
+    for (int c0 = 0; b > 1 && c0 < b; c0 += kMaxCudaCoreBatch) {
         GemvParams P;
         int64_t t = 0, end = 0;
         q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), 0x40000000LL, &P, &t, &end);
@@ -220,6 +285,23 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
                        bool pdl_first, cudaStream_t stream) {
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {calls[i].m.n, calls[i].m.k};
+    if (b == 1) {
+        q4s::Params P;
+        int grid = 0;
+        int64_t t = 0, end = 0;
+        q4_status s = plan_stream(sh, count, part_base, &P, &grid, &t, &end);
+        if (s != Q4_OK) return s;
+        for (int i = 0; i < count; ++i) {
+            P.g[i].qs = calls[i].m.qs;
+            P.g[i].d = calls[i].m.d;
+            P.g[i].x = calls[i].x;
+            P.g[i].y = calls[i].y;
+        }
+        P.ws = static_cast<uint32_t*>(ws);
+        if (cuda_failed(q4k::launch_stream(P, grid, pdl_first, stream))) return Q4_ERR_CUDA;
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return Q4_OK;
+    }
     bool pdl = pdl_first;
     for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
         const int bt = chunk_tokens(b, c0);
@@ -341,6 +423,13 @@ size_t q4_workspace_bytes(int64_t n, int64_t k, int b) {
     if (check_shape(n, k) != Q4_OK || b < 1 || b > Q4_MAX_BATCH) return 0;
     const Shape sh = {n, k};
     int64_t tmax = 0, pmax = 0;
+    if (b == 1) {
+        q4s::Params P;
+        int grid = 0;
+        int64_t t = 0, end = 0;
+        if (plan_stream(&sh, 1, 0x40000000LL, &P, &grid, &t, &end) != Q4_OK) return 0;
+        return (size_t)(part_base_for(t) + end - (int64_t)0x40000000LL);
+    }
     for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
         GemvParams P;
         int64_t t = 0, end = 0;
@@ -695,6 +784,224 @@ int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b) {
     return units_seen == P.total_units ? 0 : 33;
 }
 
+int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count) {
+    using namespace q4s;
+    if (!n || !k || count < 1 || count > Q4_MAX_GROUP) return 1;
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
+    Params P;
+    int grid = 0;
+    int64_t tickets = 0, end = 0;
+    if (plan_stream(sh, count, INT64_MAX / 4, &P, &grid, &tickets, &end) != Q4_OK) return 2;
+    const int64_t base = part_base_for(tickets);
+    if (plan_stream(sh, count, base, &P, &grid, &tickets, &end) != Q4_OK) return 2;
+    if (kSmemBytes > (int)kMaxSmem) return 3;
+    if (grid < 1 || grid > kNumSMs * Q4_STREAM_CTAS_PER_SM) return 4;
+    for (int i = 0; i < count; ++i) {
+        const Desc& G = P.g[i];
+        for (int sp = 0; sp < G.splits; ++sp)
+            if (split_blocks(G, sp) < 1 || split_blocks(G, sp) > kMaxSplitBlocks) return 5;
+    }
+    struct Tile {
+        int g, split;
+        int64_t row0;
+        int rows;
+    };
+    std::vector<std::vector<uint8_t>> cover(count);
+    for (int i = 0; i < count; ++i) cover[i].assign((size_t)(sh[i].n * (sh[i].k / Q4_QK)), 0);
+    int64_t prev_hi = 0;
+    for (int cta = 0; cta < grid; ++cta) {
+        int64_t lo, hi;
+        cta_range(P, cta, grid, &lo, &hi);
+        if (lo != prev_hi || hi < lo) return 6;
+        prev_hi = hi;
+        for (int warp = 0; warp < kWarps; ++warp) {
+            // the math loop's order: pieces, this warp's rows, tiles
+            std::vector<Tile> consumer;
+            for (int64_t pos = lo; pos < hi;) {
+                const Where w = locate(P, pos);
+                const int64_t p1 = w.seg_end < hi ? w.seg_end : hi;
+                if (p1 <= pos || w.row < 0 || w.row >= P.g[w.g].n) return 7;
+                const int64_t seg_row0 = pos - w.row;
+                int64_t ra, rb;
+                warp_rows(pos, p1, warp, &ra, &rb);
+                for (int64_t row0 = ra - seg_row0; row0 < rb - seg_row0; row0 += kRows) {
+                    const int64_t left = rb - seg_row0 - row0;
+                    consumer.push_back({w.g, w.split, row0, left < kRows ? (int)left : kRows});
+                }
+                pos = p1;
+            }
+            // the copy issuer's walk visits the same tiles in the same order
+            Walk wk;
+            wk.begin(lo, hi, warp);
+            size_t idx = 0;
+            for (bool has = wk.next_piece(P); has; has = wk.next_piece(P))
+                for (int64_t row0 = wk.wr; row0 < wk.wend; row0 += kRows, ++idx) {
+                    const int64_t left = wk.wend - row0;
+                    const int rows = left < kRows ? (int)left : kRows;
+                    if (idx >= consumer.size()) return 8;
+                    const Tile& t = consumer[idx];
+                    if (t.g != wk.g || t.split != wk.split || t.row0 != row0 || t.rows != rows) return 8;
+                }
+            if (idx != consumer.size()) return 9;
+            for (const Tile& t : consumer) {
+                const Desc& G = P.g[t.g];
+                const int kbs = split_blocks(G, t.split);
+                if (t.rows < 1 || t.rows > kRows || kbs < 1 || kbs > kMaxSplitBlocks) return 10;
+                const int64_t qs_plane = sh[t.g].n * (sh[t.g].k / 2);
+                const int64_t d_plane = round_up(sh[t.g].n * G.nb * 2, 16);
+                int64_t tx = 0;
+                // copied[b] marks the stage bytes a copy wrote, src[b] their source
+                std::vector<int64_t> src_of(kStageBytes, -1);
+                for (int lane = 0; lane < 32; ++lane) {
+                    const LaneCopy lc = lane_copy(G, t.split, t.row0, t.rows, lane);
+                    if (!lc.active) continue;
+                    const int64_t plane = lc.scales ? d_plane : qs_plane;
+                    if (lc.src_off < 0 || lc.src_off % 16 || lc.bytes % 16 || lc.bytes == 0 ||
+                        lc.src_off + lc.bytes > plane)
+                        return 11;
+                    if (lc.dst % 16 || lc.dst + lc.bytes > (uint32_t)kStageBytes) return 12;
+                    if (!lc.scales && lc.dst + lc.bytes > (uint32_t)kStageQs) return 12;
+                    if (lc.scales && lc.dst < (uint32_t)kStageQs) return 13;
+                    for (uint32_t b = 0; b < lc.bytes; ++b) {
+                        if (src_of[lc.dst + b] != -1) return 13;  // two copies overlap
+                        src_of[lc.dst + b] = (lc.scales ? (int64_t(1) << 60) : 0) + lc.src_off + b;
+                    }
+                    tx += lc.bytes;
+                }
+                if (tx >= (int64_t(1) << 20)) return 14;
+                // every byte the math reads was copied from the right place
+                for (int r = 0; r < kRows; ++r) {
+                    uint32_t qoff, doff;
+                    row_read_offsets(G, t.split, t.row0, t.rows, r, &qoff, &doff);
+                    const int rr = r < t.rows ? r : t.rows - 1;
+                    const int64_t e = (t.row0 + rr) * G.nb + (int64_t)t.split * G.nb_split;
+                    for (int j = 0; j < kbs; ++j) {
+                        for (int b = 0; b < 16; ++b)
+                            if (qoff + 16 * j + b >= (uint32_t)kStageBytes ||
+                                src_of[qoff + 16 * j + b] != (e + j) * 16 + b)
+                                return 15;
+                        for (int b = 0; b < 2; ++b)
+                            if (doff + 2 * j + b >= (uint32_t)kStageBytes ||
+                                src_of[doff + 2 * j + b] != (int64_t(1) << 60) + (e + j) * 2 + b)
+                                return 15;
+                    }
+                }
+                for (int r = 0; r < t.rows; ++r)
+                    for (int j = 0; j < kbs; ++j) {
+                        uint8_t& cv = cover[t.g][(size_t)((t.row0 + r) * G.nb +
+                                                          (int64_t)t.split * G.nb_split + j)];
+                        if (cv) return 16;
+                        cv = 1;
+                    }
+            }
+        }
+        for (int w = 0; w < kWarps; ++w)
+            for (int s = 0; s < kStages; ++s)
+                if (stage_offset(w, s) % 16 || stage_offset(w, s) + kStageBytes > (uint32_t)kSmemBytes)
+                    return 17;
+    }
+    if (prev_hi != P.total_rows) return 18;
+    for (int i = 0; i < count; ++i)
+        for (uint8_t cv : cover[i])
+            if (!cv) return 19;
+    for (int i = 0; i < count; ++i) {
+        const Desc& G = P.g[i];
+        if (G.splits < 2) continue;
+        if (G.ticket_off * 4 < q4plan::kHeaderBytes || (G.ticket_off + G.n) * 4 > base) return 20;
+        if (G.part_off * 4 < base || (G.part_off + (int64_t)G.splits * G.n) * 4 > end) return 21;
+        for (int j = i + 1; j < count; ++j) {
+            const Desc& H = P.g[j];
+            if (H.splits < 2) continue;
+            if (G.ticket_off < H.ticket_off + H.n && H.ticket_off < G.ticket_off + G.n) return 22;
+            if (G.part_off < H.part_off + (int64_t)H.splits * H.n &&
+                H.part_off < G.part_off + (int64_t)G.splits * G.n)
+                return 23;
+        }
+    }
+    return 0;
+}
+
+int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks) {
+    using namespace q4dev;
+    int64_t bad = 0;
+    // every integer in range splits into three in-range digits that add back up
+    for (int32_t X = -kXMax; X <= kXMax; ++X) {
+        int32_t a, b, c;
+        x_digits(X, &a, &b, &c);
+        if (a < -128 || a > 127 || b < -128 || b > 127 || c < -128 || c > 127 ||
+            65536 * a + 256 * b + c != X)
+            ++bad;
+    }
+    uint64_t z = seed;
+    auto next = [&]() {
+        z += 0x9E3779B97F4A7C15ull;
+        uint64_t t = z;
+        t = (t ^ (t >> 30)) * 0xBF58476D1CE4E5B9ull;
+        t = (t ^ (t >> 27)) * 0x94D049BB133111EBull;
+        return t ^ (t >> 31);
+    };
+    for (int64_t n = 0; n < blocks; ++n) {
+        float x[32];
+        uint32_t codes[32];
+        const int kind = (int)(n % 5);
+        for (int j = 0; j < 32; ++j) {
+            const uint64_t r = next();
+            const double u = ((r >> 11) & ((1ull << 40) - 1)) / double(1ull << 40) * 2.0 - 1.0;
+            double v = u;
+            if (kind == 1) v = u * ((n % 10 == 1) ? 1e-31 : 1e-20);  // tiny; below 1e-30: dropped
+            if (kind == 2) v = u * 1e30;                         // huge
+            if (kind == 3) v = (j == 7) ? 1e4 : u * 1e-3;        // one dominant element
+            if (kind == 4) v = (j % 3 == 0) ? 0.0 : u;           // exact zeros
+            x[j] = (float)v;
+            codes[j] = (uint32_t)(r >> 60);
+        }
+        if (n % 97 == 0)
+            for (int j = 0; j < 32; ++j) x[j] = 0.0f;
+        float m = 0.0f;
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
+        const float sc = xq_scale(m), inv = xq_inv(m);
+        XDigits xd;
+        int32_t sa = 0, sb = 0, sc3 = 0;
+        int32_t dig[3][32];
+        for (int j = 0; j < 32; ++j) {
+            int32_t a, b, c;
+            x_digits(xq_int(x[j], inv), &a, &b, &c);
+            dig[0][j] = a;
+            dig[1][j] = b;
+            dig[2][j] = c;
+            sa += a;
+            sb += b;
+            sc3 += c;
+        }
+        for (int w = 0; w < 8; ++w) {
+            xd.a[w] = xd.b[w] = xd.c[w] = 0u;
+            for (int m2 = 0; m2 < 4; ++m2) {
+                xd.a[w] |= (uint32_t)(uint8_t)dig[0][4 * w + m2] << (8 * m2);
+                xd.b[w] |= (uint32_t)(uint8_t)dig[1][4 * w + m2] << (8 * m2);
+                xd.c[w] |= (uint32_t)(uint8_t)dig[2][4 * w + m2] << (8 * m2);
+            }
+        }
+        // code bytes: byte j holds code j (low nibble) and code j + 16 (high nibble)
+        uint32_t qw[4] = {0u, 0u, 0u, 0u};
+        for (int j = 0; j < 16; ++j) qw[j / 4] |= (codes[j] | (codes[j + 16] << 4)) << (8 * (j % 4));
+        const float v = block_dot_int(make_uint4(qw[0], qw[1], qw[2], qw[3]), xd, -8 * sa, -8 * sb,
+                                      -8 * sc3);
+        double exact = 0.0, bound = 0.0;
+        for (int j = 0; j < 32; ++j) {
+            const double w8 = (double)codes[j] - 8.0;
+            exact += w8 * (double)x[j];
+            // half a step of s per element, plus two binary32 roundings in x * inv;
+            // a block below kXTiny is dropped whole
+            bound += fabs(w8) * (m < kXTiny ? fabs((double)x[j])
+                                            : (double)sc * 0.5000001 + fabs((double)x[j]) * 2.4e-7);
+        }
+        bound += fabs(exact) * 2.4e-7 + 1e-300;  // the binary32 result and its scaling
+        if (!(fabs((double)v * (double)sc - exact) <= bound)) ++bad;
+    }
+    return bad;
+}
+
 int64_t q4_debug_check_unpack(uint64_t seed, int64_t count) {
     int64_t bad = 0;
     auto check = [&](uint32_t word) {
@@ -731,7 +1038,7 @@ int64_t q4_debug_check_unpack(uint64_t seed, int64_t count) {
         for (int i = 0; i < 8; ++i) x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         float* xf = reinterpret_cast<float*>(x);
         xf[pos] = 1.0f;
-        const float2 r = q4dev::block_dot(q, x);
+        const float2 r = q4dev::block_dot(q, x, q4dev::unpack_consts_default());
         const int byte = (pos % 16), hi = pos >= 16;
         const uint32_t bv = (words[byte / 4] >> (8 * (byte % 4))) & 0xFFu;
         const float want = (float)((int)(hi ? (bv >> 4) : (bv & 0xFu)) - 8);

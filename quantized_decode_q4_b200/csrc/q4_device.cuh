@@ -15,6 +15,17 @@ namespace q4dev {
 // that gives up records Q4_ERR_TIMEOUT in the workspace header and the kernel
 // skips its math; copies of a few tens of KB normally land in microseconds.
 constexpr uint64_t kWaitLimitNs = 20ull * 1000 * 1000;
+// Longest a thread may sleep inside one try_wait before it re-checks the clock.
+constexpr uint32_t kSuspendHintNs = 100000;
+#ifndef Q4_WAIT_HINT
+#define Q4_WAIT_HINT 1
+#endif
+// Device unpack form: 2 = explicit PTX packing of each f32x2 pair (fewest
+// integer instructions); 0 = C++ pairs; 1 = scalar binary32. The host always
+// compiles form 0, which the host-side unpack check exercises.
+#ifndef Q4_UNPACK
+#define Q4_UNPACK 2
+#endif
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
@@ -45,18 +56,35 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // Returns true once the barrier's phase with the given parity has completed,
 // false if it did not within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+#if Q4_WAIT_HINT
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+#else
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+#endif
+    return done != 0;
+}
+
+// Returns true once the barrier's phase with the given parity has completed,
+// false if it did not within kWaitLimitNs. The clock is read only when the
+// first try did not succeed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     const uint32_t addr = smem_addr(bar);
+    if (mbar_try(addr, parity)) return true;
     const uint64_t start = global_ns();
     while (true) {
-        uint32_t done;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-            " selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
+        if (mbar_try(addr, parity)) return true;
         if (global_ns() - start > kWaitLimitNs) return false;
     }
 }
@@ -70,6 +98,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
             "r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (no completion tracking). src and
+// bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Programmatic dependent launch: let the next kernel of the stream be scheduled,
@@ -126,29 +160,119 @@ struct Pairs {
     float2 lo01, lo23, hi01, hi23;
 };
 
+__host__ __device__ __forceinline__ float2 u64_f2(uint64_t v) {
+    return f2(bits_f32((uint32_t)v), bits_f32((uint32_t)(v >> 32)));
+}
+
+// Each pair is formed by one 64-bit mask-and-OR whose two halves are single
+// 32-bit logic operations writing the two registers of the pair directly.
 __host__ __device__ __forceinline__ Pairs unpack_word(uint32_t q) {
     const uint32_t s = q >> 12;
+    const uint64_t qq = ((uint64_t)q << 32) | q;
+    const uint64_t sq = ((uint64_t)s << 32) | q;
+    const uint64_t ss = ((uint64_t)s << 32) | s;
     Pairs p;
-    p.lo01 = add2(f2(bits_f32((q & 0x0000000Fu) | 0x4B000000u),   // 2^23 + q
-                     bits_f32((q & 0x00000F00u) | 0x47000000u)),  // 2^15 + q
+    // (2^23 + q, 2^15 + q)
+    p.lo01 = add2(u64_f2((qq & 0x00000F000000000Full) | 0x470000004B000000ull),
                   f2(-8388616.0f, -32776.0f));
-    p.lo23 = add2(f2(bits_f32((q & 0x000F0000u) | 0x43000000u),   // 2^7 + q
-                     bits_f32((s & 0x0000F000u) | 0x45000000u)),  // 2^11 + q
+    // (2^7 + q, 2^11 + q)
+    p.lo23 = add2(u64_f2((sq & 0x0000F000000F0000ull) | 0x4500000043000000ull),
                   f2(-136.0f, -2056.0f));
-    p.hi01 = add2(f2(bits_f32((q & 0x000000F0u) | 0x49000000u),   // 2^19 + q
-                     bits_f32((q & 0x0000F000u) | 0x45000000u)),  // 2^11 + q
+    // (2^19 + q, 2^11 + q)
+    p.hi01 = add2(u64_f2((qq & 0x0000F000000000F0ull) | 0x4500000049000000ull),
                   f2(-524296.0f, -2056.0f));
-    p.hi23 = add2(f2(bits_f32((s & 0x00000F00u) | 0x47000000u),   // 2^15 + q
-                     bits_f32((s & 0x000F0000u) | 0x43000000u)),  // 2^7 + q
+    // (2^15 + q, 2^7 + q)
+    p.hi23 = add2(u64_f2((ss & 0x000F000000000F00ull) | 0x4300000047000000ull),
                   f2(-32776.0f, -136.0f));
     return p;
 }
 
 // Sum over one block of (q - 8) * x, with x given as 8 float4 chunks: chunk i
 // holds x[4i .. 4i+3] of the block. Returns two partial sums.
-__host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4 (&x)[8]) {
+// Constants of the register unpack: the magic exponents 2^23, 2^19, 2^15, 2^11,
+// 2^7 and the four (2^e + 8) offset pairs, as bit patterns. Kernels load them
+// once, from kernel parameters, so that they live in registers.
+struct UnpackConsts {
+    uint32_t e23, e19, e15, e11, e7;
+    unsigned long long lo01, lo23, hi01, hi23;
+};
+
+__host__ __device__ __forceinline__ UnpackConsts unpack_consts_default() {
+    UnpackConsts k;
+    k.e23 = 0x4B000000u;
+    k.e19 = 0x49000000u;
+    k.e15 = 0x47000000u;
+    k.e11 = 0x45000000u;
+    k.e7 = 0x43000000u;
+    k.lo01 = 0xC7000800CB000008ull;  // (-(2^23 + 8), -(2^15 + 8))
+    k.lo23 = 0xC5008000C3080000ull;  // (-(2^7 + 8),  -(2^11 + 8))
+    k.hi01 = 0xC5008000C9000080ull;  // (-(2^19 + 8), -(2^11 + 8))
+    k.hi23 = 0xC3080000C7000800ull;  // (-(2^15 + 8), -(2^7 + 8))
+    return k;
+}
+
+__host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4 (&x)[8],
+                                                     const UnpackConsts& k) {
     float2 acc = f2(0.0f, 0.0f);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+    (void)k;
+#if Q4_UNPACK == 1 && !defined(__CUDA_ARCH__)
+#undef Q4_UNPACK
+#define Q4_UNPACK 0
+#endif
+#if Q4_UNPACK == 1
+    // scalar form: one logic op, one add and one fused multiply-add per weight
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t v = words[w], sh = v >> 12;
+        acc.x = fmaf(__uint_as_float((v & 0xFu) | 0x4B000000u) - 8388616.0f, x[w].x, acc.x);
+        acc.y = fmaf(__uint_as_float((v & 0xF00u) | 0x47000000u) - 32776.0f, x[w].y, acc.y);
+        acc.x = fmaf(__uint_as_float((v & 0xF0000u) | 0x43000000u) - 136.0f, x[w].z, acc.x);
+        acc.y = fmaf(__uint_as_float((sh & 0xF000u) | 0x45000000u) - 2056.0f, x[w].w, acc.y);
+        acc.x = fmaf(__uint_as_float((v & 0xF0u) | 0x49000000u) - 524296.0f, x[w + 4].x, acc.x);
+        acc.y = fmaf(__uint_as_float((v & 0xF000u) | 0x45000000u) - 2056.0f, x[w + 4].y, acc.y);
+        acc.x = fmaf(__uint_as_float((sh & 0xF00u) | 0x47000000u) - 32776.0f, x[w + 4].z, acc.x);
+        acc.y = fmaf(__uint_as_float((sh & 0xF0000u) | 0x43000000u) - 136.0f, x[w + 4].w, acc.y);
+    }
+#elif Q4_UNPACK == 2 && defined(__CUDA_ARCH__)
+    // explicit PTX: each pair is packed from two logic results with mov.b64; two
+    // accumulator chains (even and odd words); the magic exponents and the pair
+    // offsets come in as registers
+    unsigned long long a[2] = {0ull, 0ull};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const unsigned long long xlo01 = ((unsigned long long)__float_as_uint(x[w].y) << 32) | __float_as_uint(x[w].x);
+        const unsigned long long xlo23 = ((unsigned long long)__float_as_uint(x[w].w) << 32) | __float_as_uint(x[w].z);
+        const unsigned long long xhi01 = ((unsigned long long)__float_as_uint(x[w + 4].y) << 32) | __float_as_uint(x[w + 4].x);
+        const unsigned long long xhi23 = ((unsigned long long)__float_as_uint(x[w + 4].w) << 32) | __float_as_uint(x[w + 4].z);
+        asm("{\n"
+            " .reg .b32 s, t0, t1;\n .reg .b64 p;\n"
+            " shr.b32 s, %1, 12;\n"
+            " lop3.b32 t0, %1, 0x0000000F, %6, 0xEA;\n"
+            " lop3.b32 t1, %1, 0x00000F00, %8, 0xEA;\n"
+            " mov.b64 p, {t0, t1};\n"
+            " add.rn.f32x2 p, p, %11;\n fma.rn.f32x2 %0, p, %2, %0;\n"
+            " lop3.b32 t0, %1, 0x000F0000, %10, 0xEA;\n"
+            " lop3.b32 t1, s, 0x0000F000, %9, 0xEA;\n"
+            " mov.b64 p, {t0, t1};\n"
+            " add.rn.f32x2 p, p, %12;\n fma.rn.f32x2 %0, p, %3, %0;\n"
+            " lop3.b32 t0, %1, 0x000000F0, %7, 0xEA;\n"
+            " lop3.b32 t1, %1, 0x0000F000, %9, 0xEA;\n"
+            " mov.b64 p, {t0, t1};\n"
+            " add.rn.f32x2 p, p, %13;\n fma.rn.f32x2 %0, p, %4, %0;\n"
+            " lop3.b32 t0, s, 0x00000F00, %8, 0xEA;\n"
+            " lop3.b32 t1, s, 0x000F0000, %10, 0xEA;\n"
+            " mov.b64 p, {t0, t1};\n"
+            " add.rn.f32x2 p, p, %14;\n fma.rn.f32x2 %0, p, %5, %0;\n"
+            "}\n"
+            : "+l"(a[w & 1])
+            : "r"(words[w]), "l"(xlo01), "l"(xlo23), "l"(xhi01), "l"(xhi23),
+              "r"(k.e23), "r"(k.e19), "r"(k.e15), "r"(k.e11), "r"(k.e7),
+              "l"(k.lo01), "l"(k.lo23), "l"(k.hi01), "l"(k.hi23));
+    }
+    acc = f2(__uint_as_float((uint32_t)a[0]) + __uint_as_float((uint32_t)a[1]),
+             __uint_as_float((uint32_t)(a[0] >> 32)) + __uint_as_float((uint32_t)(a[1] >> 32)));
+#else
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         const Pairs p = unpack_word(words[w]);
@@ -157,6 +281,7 @@ __host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4
         acc = fma2(p.hi01, f2(x[w + 4].x, x[w + 4].y), acc);
         acc = fma2(p.hi23, f2(x[w + 4].z, x[w + 4].w), acc);
     }
+#endif
     return acc;
 }
 

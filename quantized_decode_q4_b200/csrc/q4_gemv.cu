@@ -129,40 +129,57 @@ __global__ void __launch_bounds__(kThreads) gemv_b1_kernel(const __grid_constant
     // stage this split's activations in the lane-interleaved layout
     float4* xs4 = reinterpret_cast<float4*>(smem + smem_x_offset());
     const float4* xg = reinterpret_cast<const float4*>(G.x + (int64_t)u.split * G.nb_split * 32);
-    for (int c = threadIdx.x; c < kbs * 8; c += kThreads) xs4[x_slot_b1(c >> 3, c & 7)] = xg[c];
+    {
+        // all loads first, then all stores: one round trip to L2, not one per chunk
+        constexpr int kPer = (kMaxBlocksPerSplit * 8 + kThreads - 1) / kThreads;
+        float4 t[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int c = threadIdx.x + i * kThreads;
+            if (c < kbs * 8) t[i] = xg[c];
+        }
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int c = threadIdx.x + i * kThreads;
+            if (c < kbs * 8) xs4[x_slot_b1(c >> 3, c & 7)] = t[i];
+        }
+    }
     __syncthreads();
 
     if (rows > 0 && wait_rows(P, bar, lane)) {
-        uint32_t shift[kRowsPerWarp];
+        // Rows past the end of the matrix repeat the last real row (results are
+        // not stored), so the inner loop has no per-row branches.
+        const uint8_t* qrow[kRowsPerWarp];
+        const uint16_t* drow[kRowsPerWarp];
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r)
-            shift[r] = r < rows ? d_range(G, row0 + r, u.split, kbs).shift : 0u;
-        float2 acc[kRowsPerWarp];
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int rr = r < rows ? r : rows - 1;
+            qrow[r] = qsw + (size_t)rr * G.nb_split * 16 + lane * 16;
+            drow[r] = dsw + rr * P.d_slot + d_range(G, row0 + rr, u.split, kbs).shift + lane;
+        }
+        float acc[kRowsPerWarp];
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) acc[r] = f2(0.0f, 0.0f);
+        for (int r = 0; r < kRowsPerWarp; ++r) acc[r] = 0.0f;
 
+        const float4* xl = xs4 + lane;
         const int iters = (kbs + 31) >> 5;
         for (int it = 0; it < iters; ++it) {
-            const int j = (it << 5) + lane;
-            if (j < kbs) {
+            if ((it << 5) + lane < kbs) {
                 float4 xv[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) xv[i] = xs4[x_slot_b1(j, i)];
+                for (int i = 0; i < 8; ++i) xv[i] = xl[((it * 8 + i) << 5)];
 #pragma unroll
                 for (int r = 0; r < kRowsPerWarp; ++r) {
-                    if (r < rows) {
-                        const uint4 q = *reinterpret_cast<const uint4*>(
-                            qsw + ((size_t)r * G.nb_split + j) * 16);
-                        const float dd =
-                            __half2float(__ushort_as_half(dsw[r * P.d_slot + shift[r] + j]));
-                        acc[r] = fma2(block_dot(q, xv), f2(dd, dd), acc[r]);
-                    }
+                    const uint4 q = *reinterpret_cast<const uint4*>(qrow[r] + it * 512);
+                    const float dd = __half2float(__ushort_as_half(drow[r][it * 32]));
+                    const float2 b = block_dot(q, xv, unpack_consts_default());
+                    acc[r] = fmaf(dd, b.x + b.y, acc[r]);
                 }
             }
         }
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
-            const float s = warp_sum(acc[r].x + acc[r].y);
+            const float s = warp_sum(acc[r]);
             if (lane == r && r < rows) store_row(P, G, u.split, 0, row0 + r, s);
         }
     }

@@ -26,7 +26,10 @@ constexpr int kWarps = 4;                         // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerWarp = 4;                   // rows per warp (x reuse)
 constexpr int kRowsPerCta = kWarps * kRowsPerWarp;
-constexpr int kMaxBlocksPerSplit = 128;           // K per split <= 4096
+#ifndef Q4_MAX_BLOCKS_PER_SPLIT
+#define Q4_MAX_BLOCKS_PER_SPLIT 128
+#endif
+constexpr int kMaxBlocksPerSplit = Q4_MAX_BLOCKS_PER_SPLIT;  // K per split (blocks of 32)
 constexpr int kHeaderBytes = 256;                 // workspace status header
 constexpr int kBarrierBytes = 128;                // mbarriers at the start of smem
 

@@ -111,6 +111,39 @@ def test_register_unpack_on_host():
     assert q4.check_unpack(12345, 500000) == 0
 
 
+def _check_stream(shapes):
+    L = q4.lib()
+    f = L.q4_debug_check_stream
+    f.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    f.restype = ctypes.c_int
+    n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
+    k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
+    return f(n, k, len(shapes))
+
+
+def test_streaming_plans_replay_on_host():
+    """Every byte the batch-1 kernel reads was copied from the right place, every
+    (row, block) is covered once, copy issuer and math loop walk the same tiles."""
+    for s in _all_shapes() + EDGE_SHAPES + [(1000, 2080), (3, 992)]:
+        assert _check_stream([s]) == 0, s
+    for wl in synth.workloads().values():
+        groups = {}
+        for g in wl.gemvs:
+            groups.setdefault(g.group, []).append((g.n, g.k))
+        for shapes in {tuple(v) for v in groups.values()}:
+            assert _check_stream(list(shapes)) == 0, shapes
+    assert _check_stream([(5, 96), (700, 2080), (3, 4160)]) == 0
+
+
+def test_integer_block_dot_on_host():
+    """Activation digits split exactly; block sums within the stated bound."""
+    L = q4.lib()
+    f = L.q4_debug_check_intdot
+    f.argtypes = [ctypes.c_uint64, ctypes.c_int64]
+    f.restype = ctypes.c_int64
+    assert f(2024, 300000) == 0
+
+
 def test_interchange_matches_oracle():
     rng = np.random.default_rng(5)
     n, k = 7, 96
