@@ -347,7 +347,7 @@ def main():
             "roofline": {
                 "bound": "hbm", "achieved": per_gpu_alg, "peak": peak, "unit": "GB/s",
                 "frac": per_gpu_alg / peak, "traffic": traffic,
-                "kernel": "q4k::gemv_stream_kernel" if args.batch == 1 else "q4k::gemv_bs_kernel",
+                "kernel": "q4k::gemv_stream_kernel" if args.batch == 1 else "q4k::gemv_tc_kernel",
                 "peak_source": peak_src,
                 "note": ("achieved = algorithmic bytes of a step (Q4_0 weights + x + y) / step "
                          f"time; the step is {step.launches} launches of this one kernel, so "

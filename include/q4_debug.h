@@ -53,6 +53,25 @@ int64_t q4_debug_check_unpack(uint64_t seed, int64_t count);
  * the number of failures (0 when correct). */
 int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks);
 
+/* The same replay for the batched tensor-core kernel (2 <= b <= 16 tokens):
+ * every CTA's range of (tile, block) units and its walk in stages, exactly-once
+ * coverage of every (tile, block), every TMA box (16-byte aligned x coordinate,
+ * inside the code row), every activation load, the shared-memory operand rows
+ * and the MMA descriptor that addresses them, the partial-sum slot of every
+ * piece of a tile (slots 0..pieces-1, each once) and its ticket, all inside
+ * their workspace regions. Returns 0 when every check holds, otherwise the
+ * number of the first failed check (see q4_api.cu). */
+int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b);
+
+/* Check the tensor-core kernel's operand preparation on the host (the same
+ * source compiled for the CPU): the dequantised A operand of `blocks`
+ * pseudo-random code blocks holds q - 8 exactly at every MMA position, and an
+ * emulated MMA over the A words and the hi/lo B rows (written at the offsets
+ * the kernel uses, read back at the addresses the MMA descriptor gives)
+ * reproduces sum_j (q_j - 8) x_j within 2^-16 sum_j |q_j - 8| |x_j|, for both
+ * operand layouts (up to 8 tokens, and 9..16). Returns the number of failures. */
+int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks);
+
 #ifdef __cplusplus
 }
 #endif

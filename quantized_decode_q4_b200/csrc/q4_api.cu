@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <climits>
 #include <cstdint>
@@ -18,6 +19,8 @@
 #include "q4_intdot.cuh"
 #include "q4_plan.h"
 #include "q4_stream_plan.h"
+#include "q4_tc_math.cuh"
+#include "q4_tc_plan.h"
 
 namespace q4k {
 cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblocks,
@@ -28,6 +31,10 @@ cudaError_t setup_gemv_kernels(int optin_smem);
 cudaError_t launch_gemv(const q4plan::GemvParams& P, bool pdl, cudaStream_t stream);
 cudaError_t setup_stream_kernel(int optin_smem);
 cudaError_t launch_stream(const q4s::Params& P, int grid, bool pdl, cudaStream_t stream);
+cudaError_t setup_tc_kernels(int optin_smem);
+cudaError_t launch_tc(const q4t::Params& P, bool pdl, cudaStream_t stream);
+cudaError_t encode_code_map(CUtensorMap* map, const uint8_t* qs, int64_t n, int64_t k);
+int tc_tokens(int b);
 }  // namespace q4k
 
 using q4plan::GemvDesc;
@@ -48,6 +55,12 @@ bool cuda_failed(cudaError_t e) {
 // CTAs a launch aims for before K is split further: two per SM of a B200.
 constexpr int64_t kTargetUnits = 2 * 148;
 constexpr int kMaxCudaCoreBatch = 4;
+// Batches of at least this many tokens run on the tensor-core kernel; smaller
+// ones (above 1) on the CUDA-core kernel.
+#ifndef Q4_TC_MIN_BATCH
+#define Q4_TC_MIN_BATCH 2
+#endif
+constexpr int kTcMinBatch = Q4_TC_MIN_BATCH;
 constexpr uint32_t kMaxSmem = 226 * 1024;  // below the opt-in limit minus static smem
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -205,6 +218,54 @@ q4_status plan_stream(const Shape* sh, int count, int64_t part_base, q4s::Params
     return Q4_OK;
 }
 
+// Tensor-core plan over `count` GEMVs for b tokens: the flat (tile, block)
+// space, the grid, and per GEMV its partial-sum slots per tile, tickets (four
+// per tile: one per epilogue warp) and partial sums [tiles][slots][b][128].
+q4_status plan_tc(const Shape* sh, int count, int b, int64_t part_base, q4t::Params* P,
+                  int64_t* tickets, int64_t* ws_end) {
+    if (count < 1 || count > Q4_MAX_GROUP || b < 2 || b > Q4_MAX_BATCH) return Q4_ERR_INVALID_ARG;
+    std::memset(P, 0, sizeof *P);
+    int64_t F = 0;
+    for (int i = 0; i < count; ++i) {
+        q4_status s = check_shape(sh[i].n, sh[i].k);
+        if (s != Q4_OK) return s;
+        q4t::Desc& G = P->g[i];
+        G.n = sh[i].n;
+        G.nb = (int32_t)(sh[i].k / Q4_QK);
+        G.tiles = (int32_t)ceil_div(sh[i].n, q4t::kM);
+        G.flat_begin = F;
+        F += (int64_t)G.tiles * G.nb;
+        if (F >= (int64_t(1) << 31) || sh[i].k / 2 >= (int64_t(1) << 31) ||
+            sh[i].n >= (int64_t(1) << 31))
+            return Q4_ERR_INVALID_ARG;  // 32-bit unit space and TMA coordinates
+    }
+    P->count = count;
+    P->b = b;
+    P->total = F;
+    P->grid = (int32_t)std::min<int64_t>(kNumSMs, F);
+    int64_t tick = 0, part = part_base;
+    for (int i = 0; i < count; ++i) {
+        q4t::Desc& G = P->g[i];
+        int maxp = 1;
+        for (int32_t t = 0; t < G.tiles; ++t) {
+            int np = 0, slot = 0;
+            q4t::tile_pieces(*P, G, t, 0, &np, &slot);
+            maxp = std::max(maxp, np);
+        }
+        G.maxp = maxp;
+        if (maxp > 1) {
+            G.ticket_off = q4plan::kHeaderBytes / 4 + tick;
+            tick += 4 * (int64_t)G.tiles;
+            G.part_off = part / 4;
+            part += round_up((int64_t)G.tiles * maxp * b * q4t::kM * 4, 256);
+        }
+    }
+    if (q4plan::kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
+    *tickets = tick;
+    *ws_end = part;
+    return Q4_OK;
+}
+
 // Token chunks: batches above the CUDA-core kernel's width run as several
 // launches of at most kMaxCudaCoreBatch tokens.
 int chunk_tokens(int b, int c0) { return std::min(kMaxCudaCoreBatch, b - c0); }
@@ -226,6 +287,7 @@ q4_status ensure_device() {
     if (major != 10 || minor != 0) return Q4_ERR_UNSUPPORTED;
     if (cuda_failed(q4k::setup_gemv_kernels(optin))) return Q4_ERR_CUDA;
     if (cuda_failed(q4k::setup_stream_kernel(optin))) return Q4_ERR_CUDA;
+    if (cuda_failed(q4k::setup_tc_kernels(optin))) return Q4_ERR_CUDA;
     g_dev_ready[dev] = true;
     return Q4_OK;
 }
@@ -236,8 +298,45 @@ struct GemvCall {
     float* y;
 };
 
-// Validate one group for `b` tokens; returns its largest ticket count over the
-// token chunks and the partial-sum bytes it needs past the ticket region.
+// Tickets and partial-sum bytes (past the ticket region) of one launch group
+// of the given shapes for `b` tokens, planned exactly as the launch will be.
+q4_status group_need(const Shape* sh, int count, int b, int64_t* tickets, int64_t* part_bytes) {
+    if (count < 1 || count > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
+    if (b < 1 || b > Q4_MAX_BATCH) return Q4_ERR_UNSUPPORTED;
+    constexpr int64_t kBase = 0x40000000LL;
+    int64_t tmax = 0, pmax = 0;
+    if (b == 1) {
+        q4s::Params P;
+        int grid = 0;
+        int64_t t = 0, end = 0;
+        q4_status s = plan_stream(sh, count, kBase, &P, &grid, &t, &end);
+        if (s != Q4_OK) return s;
+        tmax = t;
+        pmax = end - kBase;
+    } else if (b >= kTcMinBatch) {
+        q4t::Params P;
+        int64_t t = 0, end = 0;
+        q4_status s = plan_tc(sh, count, b, kBase, &P, &t, &end);
+        if (s != Q4_OK) return s;
+        tmax = t;
+        pmax = end - kBase;
+    } else {
+        for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
+            GemvParams P;
+            int64_t t = 0, end = 0;
+            q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), kBase, &P, &t, &end);
+            if (s != Q4_OK) return s;
+            tmax = std::max(tmax, t);
+            pmax = std::max(pmax, end - kBase);
+        }
+    }
+    *tickets = tmax;
+    *part_bytes = pmax;
+    return Q4_OK;
+}
+
+// Validate one group for `b` tokens; returns its ticket count and the
+// partial-sum bytes it needs past the ticket region.
 q4_status check_group(const GemvCall* calls, int count, int b, int64_t* tickets,
                       int64_t* part_bytes) {
     if (count < 1 || count > Q4_MAX_GROUP) return Q4_ERR_INVALID_ARG;
@@ -250,27 +349,7 @@ q4_status check_group(const GemvCall* calls, int count, int b, int64_t* tickets,
         if (!aligned(calls[i].x, 16) || !aligned(calls[i].y, 16)) return Q4_ERR_MISALIGNED;
         sh[i] = {calls[i].m.n, calls[i].m.k};
     }
-    int64_t tmax = 0, pmax = 0;
-    if (b == 1) {
-        q4s::Params P;
-        int grid = 0;
-        int64_t t = 0, end = 0;
-        q4_status s = plan_stream(sh, count, 0x40000000LL, &P, &grid, &t, &end);
-        if (s != Q4_OK) return s;
-        tmax = t;
-        pmax = end - (int64_t)0x40000000LL;
-    }
-    for (int c0 = 0; b > 1 && c0 < b; c0 += kMaxCudaCoreBatch) {
-        GemvParams P;
-        int64_t t = 0, end = 0;
-        q4_status s = plan_shapes(sh, count, chunk_tokens(b, c0), 0x40000000LL, &P, &t, &end);
-        if (s != Q4_OK) return s;
-        tmax = std::max(tmax, t);
-        pmax = std::max(pmax, end - (int64_t)0x40000000LL);
-    }
-    *tickets = tmax;
-    *part_bytes = pmax;
-    return Q4_OK;
+    return group_need(sh, count, b, tickets, part_bytes);
 }
 
 q4_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -299,6 +378,25 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
         }
         P.ws = static_cast<uint32_t*>(ws);
         if (cuda_failed(q4k::launch_stream(P, grid, pdl_first, stream))) return Q4_ERR_CUDA;
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return Q4_OK;
+    }
+    if (b >= kTcMinBatch) {
+        q4t::Params P;
+        int64_t t = 0, end = 0;
+        q4_status s = plan_tc(sh, count, b, part_base, &P, &t, &end);
+        if (s != Q4_OK) return s;
+        for (int i = 0; i < count; ++i) {
+            P.g[i].qs = calls[i].m.qs;
+            P.g[i].d = calls[i].m.d;
+            P.g[i].x = calls[i].x;
+            P.g[i].y = calls[i].y;
+            if (cuda_failed(q4k::encode_code_map(&P.tmap[i], calls[i].m.qs, calls[i].m.n,
+                                                 calls[i].m.k)))
+                return Q4_ERR_CUDA;
+        }
+        P.ws = static_cast<uint32_t*>(ws);
+        if (cuda_failed(q4k::launch_tc(P, pdl_first, stream))) return Q4_ERR_CUDA;
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return Q4_OK;
     }
@@ -371,6 +469,7 @@ q4_status stack_check(const q4_stack* s, int b, std::vector<std::pair<int, int>>
 }
 
 uint64_t stack_kernel_count(const std::vector<std::pair<int, int>>& groups, int b) {
+    if (b == 1 || b >= kTcMinBatch) return (uint64_t)groups.size();
     return (uint64_t)groups.size() * (uint64_t)ceil_div(b, kMaxCudaCoreBatch);
 }
 
@@ -422,23 +521,9 @@ q4_status q4_dequant(const q4_matrix* m, float* w_out, void* stream) {
 size_t q4_workspace_bytes(int64_t n, int64_t k, int b) {
     if (check_shape(n, k) != Q4_OK || b < 1 || b > Q4_MAX_BATCH) return 0;
     const Shape sh = {n, k};
-    int64_t tmax = 0, pmax = 0;
-    if (b == 1) {
-        q4s::Params P;
-        int grid = 0;
-        int64_t t = 0, end = 0;
-        if (plan_stream(&sh, 1, 0x40000000LL, &P, &grid, &t, &end) != Q4_OK) return 0;
-        return (size_t)(part_base_for(t) + end - (int64_t)0x40000000LL);
-    }
-    for (int c0 = 0; c0 < b; c0 += kMaxCudaCoreBatch) {
-        GemvParams P;
-        int64_t t = 0, end = 0;
-        if (plan_shapes(&sh, 1, chunk_tokens(b, c0), 0x40000000LL, &P, &t, &end) != Q4_OK)
-            return 0;
-        tmax = std::max(tmax, t);
-        pmax = std::max(pmax, end - (int64_t)0x40000000LL);
-    }
-    return (size_t)(part_base_for(tmax) + pmax);
+    int64_t t = 0, p = 0;
+    if (group_need(&sh, 1, b, &t, &p) != Q4_OK) return 0;
+    return (size_t)(part_base_for(t) + p);
 }
 
 q4_status q4_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -920,6 +1005,227 @@ int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count) {
         }
     }
     return 0;
+}
+
+int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
+    using namespace q4t;
+    if (!n || !k || count < 1 || count > Q4_MAX_GROUP || b < 2 || b > Q4_MAX_BATCH) return 1;
+    Shape sh[Q4_MAX_GROUP];
+    for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
+    Params P;
+    int64_t tickets = 0, end = 0;
+    if (plan_tc(sh, count, b, INT64_MAX / 4, &P, &tickets, &end) != Q4_OK) return 2;
+    const int64_t base = part_base_for(tickets);
+    if (plan_tc(sh, count, b, base, &P, &tickets, &end) != Q4_OK) return 2;
+    if (kSmemBytes > (int)kMaxSmem || 2 * kSmemBytes <= 228 * 1024) return 3;  // one CTA per SM
+    if (P.grid < 1 || P.grid > kNumSMs || P.grid > P.total) return 4;
+    const bool split = q4k::tc_tokens(b) <= 8;
+    // operand layout: every (block, chunk, K half, MMA row) has its own 16-byte
+    // row inside the stage's activation region, and the MMA descriptor of each
+    // operand addresses exactly those rows
+    {
+        std::vector<int> used(kXBytes / 16, 0);
+        for (int i = 0; i < kS; ++i)
+            for (int c2 = 0; c2 < 2; ++c2)
+                for (int hl = 0; hl < (split ? 1 : 2); ++hl) {
+                    const uint32_t op = x_operand_off(split, i, c2, hl);
+                    for (int rho = 0; rho < kN; ++rho)
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t a = op + hh * kLBO + (rho >> 3) * kSBO + (rho & 7) * 16;
+                            if (a % 16 || a + 16 > (uint32_t)kXBytes) return 30;
+                            if (used[a / 16]++) return 31;
+                        }
+                }
+        for (int i = 0; i < kS; ++i)
+            for (int c2 = 0; c2 < 2; ++c2)
+                for (int t = 0; t < (split ? 8 : 16); ++t)
+                    for (int hh = 0; hh < 2; ++hh)
+                        for (int hl = 0; hl < 2; ++hl) {
+                            const int rho = split ? (hl ? 8 + t : t) : t;
+                            const uint32_t want = x_operand_off(split, i, c2, hl) + hh * kLBO +
+                                                  (rho >> 3) * kSBO + (rho & 7) * 16;
+                            if (x_row_off(split, i, c2, hh, t, hl) != want) return 32;
+                        }
+        const uint64_t dsc = smem_desc(0x1230u);
+        if ((dsc & 0x3FFF) != (0x1230u >> 4) || ((dsc >> 16) & 0x3FFF) != kLBO / 16 ||
+            ((dsc >> 32) & 0x3FFF) != kSBO / 16 || ((dsc >> 46) & 3) != 1 || (dsc >> 61) != 0)
+            return 33;
+        for (int st = 0; st < kStages; ++st)
+            if (stage_base(st) % 1024 || stage_d(st) + kDBytes > (uint32_t)kSmemBytes ||
+                stage_codes(st) + kCodesBytes != stage_x(st))
+                return 34;
+        if (kSlots * kSlotCols > 512) return 35;
+    }
+    std::vector<std::vector<uint8_t>> cover(count);
+    for (int i = 0; i < count; ++i)
+        cover[i].assign((size_t)P.g[i].tiles * P.g[i].nb, 0);
+    // slots seen per (GEMV, tile)
+    std::vector<std::vector<std::vector<int>>> slots(count);
+    for (int i = 0; i < count; ++i) slots[i].resize(P.g[i].tiles);
+    int64_t prev_hi = 0;
+    for (int cta = 0; cta < P.grid; ++cta) {
+        int64_t lo, hi;
+        cta_range(P.total, cta, P.grid, &lo, &hi);
+        if (lo != prev_hi || hi <= lo) return 6;
+        prev_hi = hi;
+        Walk wk;
+        wk.begin(lo, hi);
+        Stage s;
+        int64_t pos = lo;
+        bool expect_first = true;
+        int cur_g = -1;
+        int32_t cur_tile = -1, next_kb = -1;
+        while (wk.next(P, &s)) {
+            const Desc& G = P.g[s.g];
+            if (s.nblk < 1 || s.nblk > kS || s.kb0 < 0 || s.kb0 + s.nblk > G.nb) return 7;
+            if (s.tile < 0 || s.tile >= G.tiles) return 7;
+            if (G.flat_begin + (int64_t)s.tile * G.nb + s.kb0 != pos) return 8;  // contiguous
+            if (s.first != expect_first) return 9;
+            if (!s.first && (s.g != cur_g || s.tile != cur_tile || s.kb0 != next_kb)) return 9;
+            cur_g = s.g;
+            cur_tile = s.tile;
+            next_kb = s.kb0 + s.nblk;
+            pos += s.nblk;
+            for (int i = 0; i < s.nblk; ++i) {
+                uint8_t& cv = cover[s.g][(size_t)s.tile * G.nb + s.kb0 + i];
+                if (cv) return 10;
+                cv = 1;
+                // TMA box: x aligned, inside the row; first row inside the matrix
+                const int64_t x = 16 * (int64_t)(s.kb0 + i);
+                if (x % 16 || x + 16 > sh[s.g].k / 2 || (int64_t)s.tile * kM >= sh[s.g].n) return 11;
+                // activation loads inside every token's row
+                if (32 * (int64_t)(s.kb0 + i) + 32 > sh[s.g].k) return 12;
+            }
+            if (s.last) {
+                if (pos != hi && G.flat_begin + (int64_t)(s.tile + 1) * G.nb != pos) return 13;
+                int np = 0, slot = 0;
+                tile_pieces(P, G, s.tile, cta, &np, &slot);
+                if (np < 1 || np > G.maxp || slot < 0 || slot >= np) return 14;
+                if (np > 1) {
+                    const int64_t p0 = G.part_off + ((int64_t)s.tile * G.maxp + slot) * b * kM;
+                    if (p0 * 4 < base || (p0 + (int64_t)b * kM) * 4 > end) return 15;
+                    const int64_t t0 = G.ticket_off + (int64_t)s.tile * 4;
+                    if (t0 * 4 < q4plan::kHeaderBytes || (t0 + 4) * 4 > base) return 16;
+                }
+                slots[s.g][s.tile].push_back(slot);
+                expect_first = true;
+            } else {
+                expect_first = false;
+            }
+        }
+        if (pos != hi || !expect_first) return 17;
+    }
+    if (prev_hi != P.total) return 18;
+    for (int i = 0; i < count; ++i) {
+        for (uint8_t cv : cover[i])
+            if (!cv) return 19;
+        for (int32_t t = 0; t < P.g[i].tiles; ++t) {
+            std::vector<int>& v = slots[i][t];
+            std::sort(v.begin(), v.end());
+            int np = 0, slot = 0;
+            tile_pieces(P, P.g[i], t, 0, &np, &slot);
+            if ((int)v.size() != np) return 20;
+            for (int j = 0; j < np; ++j)
+                if (v[j] != j) return 20;
+        }
+    }
+    for (int i = 0; i < count; ++i) {
+        const Desc& G = P.g[i];
+        if (G.maxp < 2) continue;
+        for (int j = i + 1; j < count; ++j) {
+            const Desc& H = P.g[j];
+            if (H.maxp < 2) continue;
+            if (G.ticket_off < H.ticket_off + 4 * H.tiles && H.ticket_off < G.ticket_off + 4 * G.tiles)
+                return 22;
+            const int64_t gs = (int64_t)G.tiles * G.maxp * b * kM;
+            const int64_t hs = (int64_t)H.tiles * H.maxp * b * kM;
+            if (G.part_off < H.part_off + hs && H.part_off < G.part_off + gs) return 23;
+        }
+    }
+    return 0;
+}
+
+int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks) {
+    using namespace q4t;
+    int64_t bad = 0;
+    uint64_t st = seed ? seed : 1;
+    auto next = [&st]() {
+        st ^= st << 13;
+        st ^= st >> 7;
+        st ^= st << 17;
+        return st;
+    };
+    // element map: a bijection of 0..31
+    {
+        int seen[32] = {0};
+        for (int kap = 0; kap < 32; ++kap) {
+            const int e = element_at(kap);
+            if (e < 0 || e > 31 || seen[e]++) ++bad;
+        }
+    }
+    std::vector<uint8_t> mem(kXBytes);
+    for (int64_t it = 0; it < blocks; ++it) {
+        uint8_t codes[16];
+        for (int j = 0; j < 16; ++j) codes[j] = (uint8_t)next();
+        int q[32];
+        for (int j = 0; j < 16; ++j) {
+            q[j] = codes[j] & 15;
+            q[j + 16] = codes[j] >> 4;
+        }
+        const int mag = (int)(next() % 5);
+        const float scale = mag == 0 ? 1.0f : mag == 1 ? 1e-3f : mag == 2 ? 37.0f : mag == 3 ? 1e-20f : 3e20f;
+        float x[32];
+        for (int j = 0; j < 32; ++j) {
+            const double u = (double)(next() >> 11) * (1.0 / 9007199254740992.0);
+            x[j] = (float)((2.0 * u - 1.0) * scale);
+        }
+        uint4 qv;
+        std::memcpy(&qv, codes, 16);
+        uint32_t a[16];
+        q4tm::dequant_block(qv, a);
+        // A value at MMA position kappa: column kappa/2, half kappa%2
+        double aval[32];
+        for (int kap = 0; kap < 32; ++kap) {
+            const uint32_t bits = (a[kap >> 1] >> (16 * (kap & 1))) & 0xFFFFu;
+            aval[kap] = (double)q4tm::bf16_value(bits);
+            if (aval[kap] != (double)(q[element_at(kap)] - 8)) ++bad;
+        }
+        for (int mode = 0; mode < 2; ++mode) {
+            const bool split = mode == 0;
+            std::fill(mem.begin(), mem.end(), 0);
+            // token 0 of block 0 in the layout the x warps write
+            for (int c2 = 0; c2 < 2; ++c2)
+                for (int hh = 0; hh < 2; ++hh) {
+                    float e[8];
+                    for (int m = 0; m < 8; ++m) e[m] = x[16 * c2 + 8 * hh + m];
+                    uint4 H, L;
+                    q4tm::split_row(e, &H, &L);
+                    std::memcpy(&mem[x_row_off(split, 0, c2, hh, 0, 0)], &H, 16);
+                    std::memcpy(&mem[x_row_off(split, 0, c2, hh, 0, 1)], &L, 16);
+                }
+            // the MMA: D[row 0][col] = sum_kappa A[kappa] B[col][kappa] over both chunks
+            double dsum = 0.0;
+            for (int hl = 0; hl < 2; ++hl) {
+                const int col = split ? (hl ? 8 : 0) : 0;
+                for (int kap = 0; kap < 32; ++kap) {
+                    const int c2 = kap >> 4, kk = kap & 15;
+                    const uint32_t op = x_operand_off(split, 0, c2, split ? 0 : hl);
+                    const uint32_t addr = op + (kk >> 3) * kLBO + (col >> 3) * kSBO + (col & 7) * 16 +
+                                          (kk & 7) * 2;
+                    uint16_t bits;
+                    std::memcpy(&bits, &mem[addr], 2);
+                    dsum += aval[kap] * (double)q4tm::bf16_value(bits);
+                }
+            }
+            double exact = 0.0, bound = 0.0;
+            for (int j = 0; j < 32; ++j) {
+                exact += (double)(q[j] - 8) * (double)x[j];
+                bound += std::fabs((double)(q[j] - 8)) * std::fabs((double)x[j]);
+            }
+            if (!(std::fabs(dsum - exact) <= bound * std::ldexp(1.0, -16) + 1e-300)) ++bad;
+        }
+    }
+    return bad;
 }
 
 int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks) {

@@ -1,0 +1,595 @@
+// Batched (2..16 tokens) Q4_0 decode GEMV on the sm_100a tensor cores.
+//
+// "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
+// section 3 "Dequantizzazione Integrata": for a matrix-matrix product the
+// weights are dequantised into fast on-chip memory and reused there. Here the
+// on-chip memory is tensor memory: each 32-weight block of a 128-row tile is
+// dequantised once to (q - 8) as bf16 (exact) and written with tcgen05.st into
+// a tensor-memory slot, and tcgen05.mma multiplies it with the tokens'
+// activations held in shared memory as bf16 hi + lo parts (x = hi + lo to
+// 2^-16 relative). Every block has its own binary32 accumulator, so its binary16
+// scale is applied exactly once, by the epilogue: y[t][r] += d[r][b] * D_b[r][t].
+//
+// Roles of the 14 warps of a CTA (one CTA per SM, persistent over a contiguous
+// range of (tile, block) units):
+//   producer (1 thread)   2-D TMA loads of the code bytes, 16 B x 128 rows per block
+//   x warps (4)           activations -> bf16 hi/lo B operands, scales -> binary32
+//   dequant warps (4)     codes -> (q - 8) bf16 A operands in tensor memory
+//   MMA thread (1)        tcgen05.mma M = 128, N = 16, K = 16 (2 or 4 per block)
+//   epilogue warps (4)    tcgen05.ld of each block's accumulator, scale, sum
+// Shared-memory stages and tensor-memory slots are handed over with mbarriers;
+// every wait is bounded and a wait that gives up records Q4_ERR_TIMEOUT, makes
+// every role leave its loop, and the kernel still waits for its own copies and
+// MMAs before it frees tensor memory and returns.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "q4_device.cuh"
+#include "q4_tc_math.cuh"
+#include "q4_tc_plan.h"
+
+using namespace q4dev;
+
+namespace q4k {
+
+namespace {
+
+constexpr uint32_t kTimeoutFlag = 1u;
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_alloc(uint32_t dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive once on `bar` when every tcgen05.mma this thread issued so far is done.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// D[128 x 16] (+)= A[128 x 16] (tensor memory) * B[16 x 16]^T (shared memory)
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, {%5, %5, %5, %5}, p;\n}\n" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(q4t::kInstrDesc), "r"(0u)
+        : "memory");
+}
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+struct Ctx {
+    uint8_t* smem;
+    uint32_t sbase;  // shared-memory address of smem
+    uint32_t tmem;   // tensor-memory base (lane 0, first column)
+    int* abort_flag;
+    int64_t lo, hi;
+
+    __device__ uint32_t bar(int i) const { return sbase + 8u * (uint32_t)i; }
+    __device__ bool aborted() const { return *reinterpret_cast<volatile int*>(abort_flag) != 0; }
+    __device__ void abort(const q4t::Params& P) const {
+        *reinterpret_cast<volatile int*>(abort_flag) = 1;
+        atomicOr(P.ws, kTimeoutFlag);
+    }
+};
+
+// Bounded wait of a single thread.
+__device__ __forceinline__ bool wait1(const Ctx& C, const q4t::Params& P, int b, uint32_t parity) {
+    if (mbar_wait_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity)) return true;
+    C.abort(P);
+    return false;
+}
+
+// Bounded wait of a whole warp; the outcome is the same for every lane.
+__device__ __forceinline__ bool waitw(const Ctx& C, const q4t::Params& P, int b, uint32_t parity) {
+    const bool ok = __all_sync(0xffffffffu,
+                               mbar_wait_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity));
+    if (!ok && (threadIdx.x & 31) == 0) C.abort(P);
+    return ok;
+}
+
+__device__ __forceinline__ bool warp_aborted(const Ctx& C) {
+    return __shfl_sync(0xffffffffu, C.aborted() ? 1 : 0, 0) != 0;
+}
+
+// ---- producer: code bytes of every stage, one TMA box per block ----
+__device__ void run_producer(const Ctx& C, const q4t::Params& P) {
+    q4t::Walk wk;
+    wk.begin(C.lo, C.hi);
+    q4t::Stage s;
+    uint32_t q = 0;
+    while (!C.aborted() && wk.next(P, &s)) {
+        const int st = (int)(q % q4t::kStages);
+        const uint32_t v = q / q4t::kStages;
+        // from the second round of stages on, the wait depends on roles that
+        // wait for the previous kernel: wait for it first, so that the bounded
+        // wait measures this kernel only
+        if (q == (uint32_t)q4t::kStages) pdl_wait();
+        if (!wait1(C, P, q4t::kBarStageEmpty + st, (v & 1u) ^ 1u)) break;
+        const uint32_t full = C.bar(q4t::kBarCodesFull + st);
+        mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarCodesFull + st)),
+                              (uint32_t)s.nblk * q4t::kBlockCodeBytes);
+        const uint32_t dst = C.sbase + q4t::stage_codes(st);
+        for (int i = 0; i < s.nblk; ++i)
+            tma_load_2d(dst + (uint32_t)i * q4t::kBlockCodeBytes, &P.tmap[s.g], 16 * (s.kb0 + i),
+                        s.tile * q4t::kM, full);
+        (void)full;
+        ++q;
+    }
+    // every load issued lands before the kernel may exit: wait for the latest
+    // phase of each stage that was filled
+    const uint32_t n = q < (uint32_t)q4t::kStages ? q : (uint32_t)q4t::kStages;
+    for (uint32_t k = 0; k < n; ++k) {
+        const uint32_t qq = q - 1 - k;
+        mbar_wait_bounded(
+            reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarCodesFull + (int)(qq % q4t::kStages))),
+            (qq / q4t::kStages) & 1u);
+    }
+}
+
+// ---- x warps: activations -> hi/lo B operands, scales -> binary32 ----
+template <int BT>
+__device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
+    constexpr bool kSplit = BT <= 8;
+    constexpr int kMaxItems = (BT * q4t::kS * 4 + 127) / 128;
+    const int tid = xw * 32 + lane;  // 0..127
+    pdl_wait();                      // activations may come from the previous kernel
+    q4t::Walk wk;
+    wk.begin(C.lo, C.hi);
+    q4t::Stage s;
+    uint32_t q = 0;
+    while (!warp_aborted(C) && wk.next(P, &s)) {
+        const int st = (int)(q % q4t::kStages);
+        const uint32_t v = q / q4t::kStages;
+        if (!waitw(C, P, q4t::kBarStageEmpty + st, (v & 1u) ^ 1u)) break;
+        const q4t::Desc& G = P.g[s.g];
+        // loads first: scales of row tid, then this thread's activation rows
+        const int64_t row = (int64_t)s.tile * q4t::kM + tid;
+        uint16_t dv[q4t::kS];
+#pragma unroll
+        for (int i = 0; i < q4t::kS; ++i) dv[i] = 0;
+        if (row < G.n) {
+            const uint16_t* dr = G.d + row * G.nb + s.kb0;
+#pragma unroll
+            for (int i = 0; i < q4t::kS; ++i)
+                if (i < s.nblk) dv[i] = __ldg(dr + i);
+        }
+        const int per_t = s.nblk * 4;
+        const int items = P.b * per_t;
+        const int64_t k = (int64_t)G.nb * 32;
+        float4 xa[kMaxItems], xb[kMaxItems];
+#pragma unroll
+        for (int m = 0; m < kMaxItems; ++m) {
+            const int it = tid + 128 * m;
+            if (it < items) {
+                const int t = it / per_t, rem = it - t * per_t;
+                const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
+                const float4* src = reinterpret_cast<const float4*>(
+                    G.x + t * k + 32 * (int64_t)(s.kb0 + i) + 16 * c2 + 8 * hh);
+                xa[m] = __ldg(src);
+                xb[m] = __ldg(src + 1);
+            }
+        }
+        float* dsm = reinterpret_cast<float*>(C.smem + q4t::stage_d(st));
+#pragma unroll
+        for (int i = 0; i < q4t::kS; ++i)
+            if (i < s.nblk) dsm[i * q4t::kM + tid] = __half2float(__ushort_as_half(dv[i]));
+        uint8_t* xs = C.smem + q4t::stage_x(st);
+#pragma unroll
+        for (int m = 0; m < kMaxItems; ++m) {
+            const int it = tid + 128 * m;
+            if (it < items) {
+                const int t = it / per_t, rem = it - t * per_t;
+                const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
+                const float e[8] = {xa[m].x, xa[m].y, xa[m].z, xa[m].w,
+                                    xb[m].x, xb[m].y, xb[m].z, xb[m].w};
+                uint4 H, L;
+                q4tm::split_row(e, &H, &L);
+                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kSplit, i, c2, hh, t, 0)) = H;
+                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kSplit, i, c2, hh, t, 1)) = L;
+            }
+        }
+        // the MMA reads these operands through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(C.bar(q4t::kBarXFull + st));
+        ++q;
+    }
+}
+
+// ---- dequant warps: codes -> (q - 8) bf16 in tensor memory ----
+__device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane) {
+    const int r = dw * 32 + lane;
+    const uint32_t tlane = C.tmem + ((uint32_t)(dw * 32) << 16);
+    q4t::Walk wk;
+    wk.begin(C.lo, C.hi);
+    q4t::Stage s;
+    uint32_t q = 0, j = 0;
+    while (!warp_aborted(C) && wk.next(P, &s)) {
+        const int st = (int)(q % q4t::kStages);
+        const uint32_t v = q / q4t::kStages;
+        if (q == (uint32_t)(q4t::kSlots / q4t::kS)) pdl_wait();  // slots now wait for the epilogue
+        if (!waitw(C, P, q4t::kBarCodesFull + st, v & 1u)) break;
+        const uint8_t* codes = C.smem + q4t::stage_codes(st) + r * 16;
+        bool ok = true;
+        const uint32_t j0 = j;
+        for (int i = 0; i < s.nblk; ++i) {
+            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
+            if (!waitw(C, P, q4t::kBarSlotEmpty + (int)p, (u & 1u) ^ 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint4 qv = *reinterpret_cast<const uint4*>(codes + i * q4t::kBlockCodeBytes);
+            uint32_t a[16];
+            q4tm::dequant_block(qv, a);
+            tc_st16(tlane + p * q4t::kSlotCols, a);
+            ++j;
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (!ok) break;
+        if (lane == 0) {
+            for (uint32_t jj = j0; jj < j; ++jj)
+                mbar_arrive(C.bar(q4t::kBarAFull + (int)(jj % q4t::kSlots)));
+            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
+        }
+        ++q;
+    }
+}
+
+// ---- MMA thread ----
+template <int BT>
+__device__ void run_mma(const Ctx& C, const q4t::Params& P) {
+    constexpr bool kSplit = BT <= 8;
+    pdl_wait();  // the activations come after the previous kernel
+    q4t::Walk wk;
+    wk.begin(C.lo, C.hi);
+    q4t::Stage s;
+    uint32_t q = 0, j = 0;
+    while (!C.aborted() && wk.next(P, &s)) {
+        const int st = (int)(q % q4t::kStages);
+        const uint32_t v = q / q4t::kStages;
+        if (!wait1(C, P, q4t::kBarXFull + st, v & 1u)) break;
+        const uint32_t xs = C.sbase + q4t::stage_x(st);
+        bool ok = true;
+        for (int i = 0; i < s.nblk; ++i) {
+            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
+            if (!wait1(C, P, q4t::kBarAFull + (int)p, u & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a = C.tmem + p * q4t::kSlotCols;
+            const uint32_t d = a + 16;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                if (kSplit) {
+                    tc_mma(d, a + 8 * c2, q4t::smem_desc(xs + q4t::x_operand_off(true, i, c2, 0)),
+                           c2 != 0);
+                } else {
+#pragma unroll
+                    for (int hl = 0; hl < 2; ++hl)
+                        tc_mma(d, a + 8 * c2,
+                               q4t::smem_desc(xs + q4t::x_operand_off(false, i, c2, hl)),
+                               (c2 | hl) != 0);
+                }
+            }
+            tc_commit(C.bar(q4t::kBarDFull + (int)p));
+            ++j;
+        }
+        if (!ok) break;
+        tc_commit(C.bar(q4t::kBarStageEmpty + st));
+        ++q;
+    }
+    // every MMA issued completes before tensor memory is freed
+    tc_commit(C.bar(q4t::kBarDone));
+    mbar_wait_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * q4t::kBarDone), 0);
+}
+
+// ---- epilogue warps ----
+template <int BT>
+__device__ __forceinline__ void finish_piece(const q4t::Params& P, const q4t::Stage& s, int ew,
+                                             int lane, const float (&acc)[BT]) {
+    const q4t::Desc& G = P.g[s.g];
+    const int r = ew * 32 + lane;
+    const int64_t row = (int64_t)s.tile * q4t::kM + r;
+    int np, slot;
+    q4t::tile_pieces(P, G, s.tile, blockIdx.x, &np, &slot);
+    if (np == 1) {
+        if (row < G.n) {
+#pragma unroll
+            for (int t = 0; t < BT; ++t)
+                if (t < P.b) G.y[t * G.n + row] = acc[t];
+        }
+        return;
+    }
+    float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
+    float* mine = part + ((int64_t)s.tile * G.maxp + slot) * P.b * q4t::kM + r;
+#pragma unroll
+    for (int t = 0; t < BT; ++t)
+        if (t < P.b) mine[t * q4t::kM] = acc[t];
+    __threadfence();
+    __syncwarp();
+    uint32_t tk = 0;
+    uint32_t* ticket = P.ws + G.ticket_off + (int64_t)s.tile * 4 + ew;
+    if (lane == 0) tk = atomicAdd(ticket, 1u);
+    tk = __shfl_sync(0xffffffffu, tk, 0);
+    if (tk != (uint32_t)np - 1u) return;
+    __threadfence();
+    const float* base = part + (int64_t)s.tile * G.maxp * P.b * q4t::kM + r;
+#pragma unroll
+    for (int t = 0; t < BT; ++t) {
+        if (t < P.b) {
+            float sum = 0.0f;
+            for (int sl = 0; sl < np; ++sl) sum += __ldcg(base + ((int64_t)sl * P.b + t) * q4t::kM);
+            if (row < G.n) G.y[t * G.n + row] = sum;
+        }
+    }
+    if (lane == 0) *ticket = 0u;
+}
+
+template <int BT>
+__device__ void run_epilogue(const Ctx& C, const q4t::Params& P, int ew, int lane) {
+    constexpr bool kSplit = BT <= 8;
+    const int r = ew * 32 + lane;
+    const uint32_t tlane = C.tmem + ((uint32_t)(ew * 32) << 16);
+    pdl_wait();  // partial sums, tickets and y are written below
+    q4t::Walk wk;
+    wk.begin(C.lo, C.hi);
+    q4t::Stage s;
+    uint32_t q = 0, j = 0;
+    float acc[BT];
+#pragma unroll
+    for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
+    while (!warp_aborted(C) && wk.next(P, &s)) {
+        const int st = (int)(q % q4t::kStages);
+        const uint32_t v = q / q4t::kStages;
+        if (s.first) {
+#pragma unroll
+            for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
+        }
+        if (!waitw(C, P, q4t::kBarXFull + st, v & 1u)) break;  // scales of the stage
+        const float* dsm = reinterpret_cast<const float*>(C.smem + q4t::stage_d(st)) + r;
+        bool ok = true;
+        for (int i = 0; i < s.nblk; ++i) {
+            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
+            if (!waitw(C, P, q4t::kBarDFull + (int)p, u & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t D[16];
+            tc_ld16(tlane + p * q4t::kSlotCols + 16, D);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(C.bar(q4t::kBarSlotEmpty + (int)p));
+            const float dd = dsm[i * q4t::kM];
+#pragma unroll
+            for (int t = 0; t < BT; ++t) {
+                const float val = kSplit ? __uint_as_float(D[t]) + __uint_as_float(D[8 + t])
+                                         : __uint_as_float(D[t]);
+                acc[t] = fmaf(dd, val, acc[t]);
+            }
+            ++j;
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
+        ++q;
+        if (s.last) finish_piece<BT>(P, s, ew, lane, acc);
+    }
+}
+
+}  // namespace
+
+template <int BT>
+__global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_constant__ q4t::Params P) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Ctx C;
+    C.smem = smem_raw;
+    C.sbase = smem_addr(smem_raw);
+    C.abort_flag = reinterpret_cast<int*>(smem_raw + q4t::kAbortOff);
+    q4t::cta_range(P.total, blockIdx.x, P.grid, &C.lo, &C.hi);
+
+    if (threadIdx.x == 0) {
+        uint64_t* b = reinterpret_cast<uint64_t*>(smem_raw);
+        for (int st = 0; st < q4t::kStages; ++st) {
+            mbar_init(b + q4t::kBarCodesFull + st, 1);
+            mbar_init(b + q4t::kBarXFull + st, q4t::kArrivalsXFull);
+            mbar_init(b + q4t::kBarStageEmpty + st, q4t::kArrivalsStageEmpty);
+        }
+        for (int p = 0; p < q4t::kSlots; ++p) {
+            mbar_init(b + q4t::kBarAFull + p, q4t::kArrivalsAFull);
+            mbar_init(b + q4t::kBarDFull + p, 1);
+            mbar_init(b + q4t::kBarSlotEmpty + p, q4t::kArrivalsSlotEmpty);
+        }
+        mbar_init(b + q4t::kBarDone, 1);
+        *C.abort_flag = 0;
+        mbar_fence_init();
+    }
+    // operand rows of absent tokens stay zero for the whole launch
+    for (int st = 0; st < q4t::kStages; ++st)
+        for (int off = threadIdx.x * 16; off < q4t::kXBytes; off += q4t::kThreads * 16)
+            *reinterpret_cast<uint4*>(smem_raw + q4t::stage_x(st) + off) = make_uint4(0, 0, 0, 0);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 0) {
+        tc_alloc(C.sbase + q4t::kTmemAddrOff, q4t::kTmemCols);
+        tc_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    C.tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + q4t::kTmemAddrOff);
+
+    pdl_launch_dependents();
+
+    if (warp < q4t::kEpiWarp0) {
+        run_dequant(C, P, warp - q4t::kDequantWarp0, lane);
+    } else if (warp < q4t::kXWarp0) {
+        run_epilogue<BT>(C, P, warp - q4t::kEpiWarp0, lane);
+    } else if (warp < q4t::kProdWarp) {
+        run_x<BT>(C, P, warp - q4t::kXWarp0, lane);
+    } else if (warp == q4t::kProdWarp) {
+        if (lane == 0) run_producer(C, P);
+        __syncwarp();
+    } else {
+        if (lane == 0) run_mma<BT>(C, P);
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(C.tmem, q4t::kTmemCols);
+    }
+}
+
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_encode_mu;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+    std::lock_guard<std::mutex> lock(g_encode_mu);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
+                cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return nullptr;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return g_encode;
+}
+
+template <int BT>
+cudaError_t setup_one(int optin_smem) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_tc_kernel<BT>);
+    if (e != cudaSuccess) return e;
+    if (q4t::kSmemBytes + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
+    return cudaFuncSetAttribute(gemv_tc_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                q4t::kSmemBytes);
+}
+
+template <int BT>
+cudaError_t launch_one(const q4t::Params& P, bool pdl, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P.grid, 1, 1);
+    cfg.blockDim = dim3(q4t::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = q4t::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<BT>, P);
+}
+
+}  // namespace
+
+// Tensor map of the code plane of an n x k matrix: uint8 [n][k/2], box of
+// 16 bytes (one block) x 128 rows, no swizzle; rows past n read as zero.
+cudaError_t encode_code_map(CUtensorMap* map, const uint8_t* qs, int64_t n, int64_t k) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n};
+    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    const cuuint32_t box[2] = {16u, (cuuint32_t)q4t::kM};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(qs), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Token count a launch is compiled for: the smallest of 2, 4, 8, 16 >= b.
+int tc_tokens(int b) { return b <= 2 ? 2 : b <= 4 ? 4 : b <= 8 ? 8 : 16; }
+
+cudaError_t setup_tc_kernels(int optin_smem) {
+    cudaError_t e;
+    if ((e = setup_one<2>(optin_smem)) != cudaSuccess) return e;
+    if ((e = setup_one<4>(optin_smem)) != cudaSuccess) return e;
+    if ((e = setup_one<8>(optin_smem)) != cudaSuccess) return e;
+    return setup_one<16>(optin_smem);
+}
+
+cudaError_t launch_tc(const q4t::Params& P, bool pdl, cudaStream_t stream) {
+    switch (tc_tokens(P.b)) {
+        case 2: return launch_one<2>(P, pdl, stream);
+        case 4: return launch_one<4>(P, pdl, stream);
+        case 8: return launch_one<8>(P, pdl, stream);
+        default: return launch_one<16>(P, pdl, stream);
+    }
+}
+
+}  // namespace q4k

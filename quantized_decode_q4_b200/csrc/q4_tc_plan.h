@@ -1,0 +1,233 @@
+// Work decomposition and shared-memory / tensor-memory layout of the batched
+// (2..16 tokens) tensor-core GEMV, shared by the device code and by the host
+// replay in q4_debug_check_tc.
+//
+// A launch covers one dependency group (up to Q4_MAX_GROUP GEMVs). The unit of
+// work is one K block (32 weights) of one M tile (128 rows) of one GEMV. Units
+// are ordered (GEMV, tile, block) and laid end to end in one "flat" space of F
+// units; CTA c of G owns units [F c / G, F (c + 1) / G). The part of a CTA's
+// range inside one tile is a piece; a piece is walked in stages of up to kS
+// blocks. A tile covered by several pieces (several CTAs) is finished by the
+// last one to arrive: each piece stores its 128 x b partial sums in its own
+// slot (slot = CTA index - first CTA of the tile), and the last arriver adds
+// the slots in order (deterministic).
+//
+// Per stage, shared memory holds the code bytes of the stage's blocks (block i
+// at codes + 2048 i, row r at + 16 r: one 2-D TMA box of 16 bytes x 128 rows per
+// block), the activations as the MMA's B operand (bf16 hi and lo parts, in the
+// canonical K-major layout without swizzle: 8 x 16-byte core matrices) and the
+// blocks' scales as binary32 (d[i][r]).
+//
+// Tensor memory (512 columns x 128 lanes) holds kSlots slots of 32 columns, one
+// per block in flight: columns [0, 16) are the A operand (row r = lane r, the
+// block's 32 values of (q - 8) as bf16 pairs), columns [16, 32) the block's
+// accumulator D (128 x 16, binary32).
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "../../include/q4.h"
+
+#if defined(__CUDACC__)
+#define Q4T_HD __host__ __device__ __forceinline__
+#else
+#define Q4T_HD inline
+#endif
+
+namespace q4t {
+
+#ifndef Q4_TC_STAGES
+#define Q4_TC_STAGES 5
+#endif
+#ifndef Q4_TC_STAGE_BLOCKS
+#define Q4_TC_STAGE_BLOCKS 8
+#endif
+
+constexpr int kM = 128;                 // rows per tile (MMA M)
+constexpr int kN = 16;                  // MMA N
+constexpr int kS = Q4_TC_STAGE_BLOCKS;  // K blocks per stage
+constexpr int kStages = Q4_TC_STAGES;   // shared-memory ring depth
+constexpr int kSlots = 16;              // tensor-memory slots
+constexpr int kSlotCols = 32;
+constexpr int kTmemCols = kSlots * kSlotCols;  // 512
+constexpr int kBlockCodeBytes = kM * 16;       // 2048
+constexpr int kBlockXBytes = 2048;             // 2 chunks x (hi, lo) x 512 B
+constexpr int kCodesBytes = kS * kBlockCodeBytes;
+constexpr int kXBytes = kS * kBlockXBytes;
+constexpr int kDBytes = kS * kM * 4;
+constexpr int kStageBytes = kCodesBytes + kXBytes + kDBytes;
+constexpr int kHeaderBytes = 1024;  // barriers, tensor-memory address, ticket broadcast
+constexpr int kSmemBytes = kHeaderBytes + kStages * kStageBytes;
+
+// warp roles
+constexpr int kDequantWarp0 = 0;  // 4 warps: codes -> (q - 8) bf16 into tensor memory
+constexpr int kEpiWarp0 = 4;      // 4 warps: accumulators x scale, partial sums, y
+constexpr int kXWarp0 = 8;        // 4 warps: activations -> bf16 hi/lo, scales -> binary32
+constexpr int kProdWarp = 12;     // 1 thread: TMA loads of the code bytes
+constexpr int kMmaWarp = 13;      // 1 thread: tcgen05.mma issue
+constexpr int kWarps = 14;
+constexpr int kThreads = kWarps * 32;
+
+static_assert(kS >= 1 && kS <= kSlots, "stage size");
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+
+// barrier indices (uint64 words at the start of shared memory)
+constexpr int kBarCodesFull = 0;                       // [kStages]
+constexpr int kBarXFull = kBarCodesFull + kStages;     // [kStages]
+constexpr int kBarStageEmpty = kBarXFull + kStages;    // [kStages]
+constexpr int kBarAFull = kBarStageEmpty + kStages;    // [kSlots]
+constexpr int kBarDFull = kBarAFull + kSlots;          // [kSlots]
+constexpr int kBarSlotEmpty = kBarDFull + kSlots;      // [kSlots]
+constexpr int kBarDone = kBarSlotEmpty + kSlots;       // 1
+constexpr int kNumBars = kBarDone + 1;
+constexpr int kTmemAddrOff = 8 * kNumBars;            // uint32 written by tcgen05.alloc
+constexpr int kTicketOff = kTmemAddrOff + 4;          // uint32 ticket broadcast
+constexpr int kAbortOff = kTicketOff + 4;             // int32 abort flag
+static_assert(kAbortOff + 4 <= kHeaderBytes, "header");
+
+// arrivals per barrier phase
+constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 1;  // dequant warps, epilogue warps, MMA commit
+constexpr uint32_t kArrivalsXFull = 4;               // x warps
+constexpr uint32_t kArrivalsAFull = 4;               // dequant warps
+constexpr uint32_t kArrivalsSlotEmpty = 4;           // epilogue warps
+
+Q4T_HD uint32_t stage_base(int st) { return (uint32_t)(kHeaderBytes + st * kStageBytes); }
+Q4T_HD uint32_t stage_codes(int st) { return stage_base(st); }
+Q4T_HD uint32_t stage_x(int st) { return stage_base(st) + kCodesBytes; }
+Q4T_HD uint32_t stage_d(int st) { return stage_base(st) + kCodesBytes + kXBytes; }
+
+// Byte offset, inside a stage's activation region, of the 16-byte row holding
+// MMA positions [8 hh, 8 hh + 8) of chunk c2 (16 K values) of block i for MMA
+// row `row` (0..15) of operand part `hl` (0 = hi, 1 = lo). With at most 8
+// tokens (split) the hi parts of tokens t are rows t and the lo parts rows
+// 8 + t of one 16-row operand (1 KB per block); with more tokens the hi and lo
+// parts are two 16-row operands (2 KB per block) accumulated into the same D.
+// Inside one 16 x 16 operand: core matrix (row group g = row / 8, K half hh) at
+// hh * 256 + g * 128, row r % 8 at 16 (r % 8).
+constexpr uint32_t kLBO = 256;  // between the two K halves of an operand
+constexpr uint32_t kSBO = 128;  // between the two 8-row groups
+Q4T_HD uint32_t x_operand_off(bool split, int i, int c2, int hl) {
+    return split ? (uint32_t)(i * 1024 + c2 * 512)
+                 : (uint32_t)(i * 2048 + c2 * 1024 + hl * 512);
+}
+Q4T_HD uint32_t x_row_off(bool split, int i, int c2, int hh, int t, int hl) {
+    const int row = split ? (hl ? 8 + t : t) : t;
+    return x_operand_off(split, i, c2, hl) + (uint32_t)(hh * kLBO) + (uint32_t)((row >> 3) * kSBO) +
+           (uint32_t)((row & 7) * 16);
+}
+
+// Element of a block (0..31) at MMA position kappa (0..31) of the A and B
+// operands. The dequant writes tensor-memory column c = kappa / 2 (half
+// kappa % 2) of a block from its code bytes as: column 2 i + s of chunk h2
+// (= columns 8 h2 + 2 i + s) holds the nibble h2 (low / high) of bytes
+// 4 i + s (low half) and 4 i + s + 2 (high half). So element
+// 16 h2 + 4 i + s + 2 h sits at position 16 h2 + 4 i + 2 s + h.
+Q4T_HD int element_at(int kappa) {
+    const int h2 = kappa >> 4, i = (kappa >> 2) & 3, s = (kappa >> 1) & 1, h = kappa & 1;
+    return 16 * h2 + 4 * i + s + 2 * h;
+}
+
+// tcgen05.mma instruction descriptor: kind::f16, A and B bf16, D binary32,
+// both K-major, M = 128, N = 16.
+constexpr uint32_t kInstrDesc = (1u << 4)            // D format F32
+                                | (1u << 7)          // A format BF16
+                                | (1u << 10)         // B format BF16
+                                | ((uint32_t)(kN >> 3) << 17)
+                                | ((uint32_t)(kM >> 4) << 24);
+
+// Shared-memory matrix descriptor of one 16 x 16 bf16 B operand at byte
+// address `addr` (canonical K-major layout, no swizzle).
+Q4T_HD uint64_t smem_desc(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((kLBO >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((kSBO >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+struct Desc {
+    const uint8_t* qs;
+    const uint16_t* d;
+    const float* x;
+    float* y;
+    int64_t n;
+    int32_t nb;          // k / 32
+    int32_t tiles;       // ceil(n / 128)
+    int64_t flat_begin;  // first unit of this GEMV in the flat space
+    int64_t part_off;    // floats: partial sums [tiles][maxp][b][128]
+    int64_t ticket_off;  // uint32: one ticket per tile
+    int32_t maxp;        // partial slots per tile (1: no split tiles)
+    int32_t pad_;
+};
+
+struct Params {
+    CUtensorMap tmap[Q4_MAX_GROUP];  // code bytes of GEMV g: uint8 [n][k/2], box 16 x 128
+    Desc g[Q4_MAX_GROUP];
+    int32_t count;
+    int32_t b;        // tokens
+    int64_t total;    // F, < 2^31
+    int32_t grid;     // G
+    int32_t pad_;
+    uint32_t* ws;
+};
+
+// CTA owning flat unit f.
+Q4T_HD int owner(int64_t f, int64_t F, int G) { return (int)(((f + 1) * G - 1) / F); }
+
+Q4T_HD void cta_range(int64_t F, int c, int G, int64_t* lo, int64_t* hi) {
+    *lo = F * c / G;
+    *hi = F * (c + 1) / G;
+}
+
+// One stage of a CTA's walk.
+struct Stage {
+    int g;
+    int32_t tile;
+    int32_t kb0;    // first block
+    int32_t nblk;   // blocks (1..kS)
+    bool first;     // first stage of a piece
+    bool last;      // last stage of a piece
+};
+
+struct Walk {
+    int64_t pos, hi;
+    bool fresh;
+
+    Q4T_HD void begin(int64_t lo, int64_t hi_) {
+        pos = lo;
+        hi = hi_;
+        fresh = true;
+    }
+
+    Q4T_HD bool next(const Params& P, Stage* s) {
+        if (pos >= hi) return false;
+        int g = 0;
+        while (g + 1 < P.count && pos >= P.g[g + 1].flat_begin) ++g;
+        const Desc& G = P.g[g];
+        const uint32_t local = (uint32_t)(pos - G.flat_begin);
+        const uint32_t nb = (uint32_t)G.nb;
+        const uint32_t tile = local / nb;
+        const int32_t kb = (int32_t)(local - tile * nb);
+        const int64_t tile_end = G.flat_begin + (int64_t)(tile + 1) * nb;
+        const int64_t pend = tile_end < hi ? tile_end : hi;
+        const int64_t left = pend - pos;
+        s->g = g;
+        s->tile = (int32_t)tile;
+        s->kb0 = kb;
+        s->nblk = (int32_t)(left < kS ? left : kS);
+        s->first = fresh;
+        s->last = pos + s->nblk == pend;
+        pos += s->nblk;
+        fresh = s->last;
+        return true;
+    }
+};
+
+// Pieces of tile `tile` of GEMV G and the slot of CTA c among them.
+Q4T_HD void tile_pieces(const Params& P, const Desc& G, int32_t tile, int c, int* np, int* slot) {
+    const int64_t f0 = G.flat_begin + (int64_t)tile * G.nb;
+    const int64_t f1 = f0 + G.nb - 1;
+    const int c0 = owner(f0, P.total, P.grid), c1 = owner(f1, P.total, P.grid);
+    *np = c1 - c0 + 1;
+    *slot = c - c0;
+}
+
+}  // namespace q4t

@@ -136,9 +136,18 @@ def test_gemv_batched_every_output(shape, b):
     _run_full(*shape, b=b)
 
 
+@pytest.mark.parametrize("b", [2, 6, 9, 12, 16])
+@pytest.mark.parametrize("shape", [(127, 32), (129, 64), (128, 8192), (2048, 256), (300, 960),
+                                   (1000, 2080), (5, 14336)])
+def test_gemv_tensor_core_every_output(shape, b):
+    """Ragged last tiles, one-block rows, tiles split over many CTAs, every
+    compiled token width (2, 4, 8, 16) with absent tokens."""
+    _run_full(*shape, b=b)
+
+
 @pytest.mark.parametrize("shape", [s for s in _all_workload_shapes()
                                    if s[0] * s[1] > FULL_CHECK_LIMIT])
-@pytest.mark.parametrize("b", [1, 4])
+@pytest.mark.parametrize("b", [1, 4, 16])
 def test_gemv_full_size_sampled_rows(shape, b):
     n, k = shape
     seed, stream = 31, 2 * (n + k)
@@ -187,8 +196,8 @@ def test_launch_counter_counts_kernels():
     x = torch.randn(256, device="cuda")
     c0 = q4.launch_count()
     q4.gemv(m, x)
-    q4.gemv_batched(m, torch.randn(6, 256, device="cuda"))  # 4 + 2 tokens: two launches
-    assert q4.launch_count() - c0 == 3
+    q4.gemv_batched(m, torch.randn(6, 256, device="cuda"))  # one tensor-core launch
+    assert q4.launch_count() - c0 == 2
 
 
 def test_workspace_shared_by_different_shapes():

@@ -35,7 +35,8 @@ def check_step(step: DecodeStep, rows_per_gemv: int, seed: int):
 @pytest.mark.parametrize("name,b", [("single_768", 1), ("minimind_26m", 1), ("minimind_26m", 2),
                                     ("minimind_26m", 8), ("minimind_26m", 16),
                                     ("smollm2_135m", 1), ("gpt2_124m", 1),
-                                    ("smollm2_360m", 1), ("smollm2_360m", 4)])
+                                    ("smollm2_360m", 1), ("smollm2_360m", 4),
+                                    ("smollm2_135m", 12)])
 def test_stack_parity(name, b):
     step = DecodeStep(synth.workloads()[name], b)
     step.run()
@@ -43,8 +44,9 @@ def test_stack_parity(name, b):
     check_step(step, 6, 100)
 
 
-def test_graph_replay_matches_direct_launch():
-    step = DecodeStep(synth.workloads()["smollm2_135m"], 1)
+@pytest.mark.parametrize("b", [1, 16])
+def test_graph_replay_matches_direct_launch(b):
+    step = DecodeStep(synth.workloads()["smollm2_135m"], b)
     step.run()
     torch.cuda.synchronize()
     direct = [y.clone() for y in step.ys]
@@ -61,7 +63,7 @@ def test_graph_replay_matches_direct_launch():
     g.close()
 
 
-@pytest.mark.parametrize("b", [1, 4])
+@pytest.mark.parametrize("b", [1, 4, 16])
 def test_8b_class_stack_full_size(b):
     """The benchmark's workload and launch configuration, full size, sampled rows."""
     step = DecodeStep(synth.workloads()["llama8b_class"], b)

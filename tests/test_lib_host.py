@@ -135,6 +135,46 @@ def test_streaming_plans_replay_on_host():
     assert _check_stream([(5, 96), (700, 2080), (3, 4160)]) == 0
 
 
+def _check_tc(shapes, b):
+    L = q4.lib()
+    f = L.q4_debug_check_tc
+    f.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), ctypes.c_int,
+                  ctypes.c_int]
+    f.restype = ctypes.c_int
+    n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
+    k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
+    return f(n, k, len(shapes), b)
+
+
+def test_tensor_core_plans_replay_on_host():
+    """Every (tile, block) of the batched kernel is covered once, every TMA box
+    and operand row is in bounds, every split tile's pieces take slots 0..p-1."""
+    extra = [(127, 32), (129, 64), (128, 8192), (2048, 256), (1000, 2080), (5, 14336),
+             (128256, 4096)]
+    for s in _all_shapes() + EDGE_SHAPES + extra:
+        for b in (2, 3, 8, 9, 16):
+            assert _check_tc([s], b) == 0, (s, b)
+    for wl in synth.workloads().values():
+        groups = {}
+        for g in wl.gemvs:
+            groups.setdefault(g.group, []).append((g.n, g.k))
+        for shapes in {tuple(v) for v in groups.values()}:
+            for b in (2, 16):
+                assert _check_tc(list(shapes), b) == 0, (shapes, b)
+    assert _check_tc([(5, 96), (700, 2080), (3, 4160)], 4) == 0
+    assert _check_tc([(5, 96)], 1) != 0 and _check_tc([(5, 96)], 17) != 0
+
+
+def test_tensor_core_operands_on_host():
+    """The dequantised A operand is q - 8 exactly at every MMA position and an
+    emulated MMA over the staged hi/lo activations gives the block sum."""
+    L = q4.lib()
+    f = L.q4_debug_check_tc_operands
+    f.argtypes = [ctypes.c_uint64, ctypes.c_int64]
+    f.restype = ctypes.c_int64
+    assert f(77, 100000) == 0
+
+
 def test_integer_block_dot_on_host():
     """Activation digits split exactly; block sums within the stated bound."""
     L = q4.lib()
