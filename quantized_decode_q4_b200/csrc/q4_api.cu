@@ -33,7 +33,8 @@ cudaError_t setup_stream_kernel(int optin_smem);
 cudaError_t launch_stream(const q4s::Params& P, int grid, bool pdl, cudaStream_t stream);
 cudaError_t setup_tc_kernels(int optin_smem);
 cudaError_t launch_tc(const q4t::Params& P, bool pdl, cudaStream_t stream);
-cudaError_t encode_code_map(CUtensorMap* map, const uint8_t* qs, int64_t n, int64_t k);
+cudaError_t encode_tc_maps(q4t::Maps* maps, int32_t* d_box, const uint8_t* qs, const uint16_t* d,
+                           const float* x, int64_t n, int64_t k, int b);
 int tc_tokens(int b);
 }  // namespace q4k
 
@@ -233,6 +234,7 @@ q4_status plan_tc(const Shape* sh, int count, int b, int64_t part_base, q4t::Par
         G.n = sh[i].n;
         G.nb = (int32_t)(sh[i].k / Q4_QK);
         G.tiles = (int32_t)ceil_div(sh[i].n, q4t::kM);
+        G.d_box = G.nb % 8 == 0 ? 1 : 0;
         G.flat_begin = F;
         F += (int64_t)G.tiles * G.nb;
         if (F >= (int64_t(1) << 31) || sh[i].k / 2 >= (int64_t(1) << 31) ||
@@ -391,8 +393,9 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
             P.g[i].d = calls[i].m.d;
             P.g[i].x = calls[i].x;
             P.g[i].y = calls[i].y;
-            if (cuda_failed(q4k::encode_code_map(&P.tmap[i], calls[i].m.qs, calls[i].m.n,
-                                                 calls[i].m.k)))
+            if (cuda_failed(q4k::encode_tc_maps(&P.maps[i], &P.g[i].d_box, calls[i].m.qs,
+                                                calls[i].m.d, calls[i].x, calls[i].m.n,
+                                                calls[i].m.k, b)))
                 return Q4_ERR_CUDA;
         }
         P.ws = static_cast<uint32_t*>(ws);
@@ -1024,7 +1027,7 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
     // row inside the stage's activation region, and the MMA descriptor of each
     // operand addresses exactly those rows
     {
-        std::vector<int> used(kXBytes / 16, 0);
+        std::vector<int> used(kXOpBytes / 16, 0);
         for (int i = 0; i < kS; ++i)
             for (int c2 = 0; c2 < 2; ++c2)
                 for (int hl = 0; hl < (split ? 1 : 2); ++hl) {
@@ -1032,7 +1035,7 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
                     for (int rho = 0; rho < kN; ++rho)
                         for (int hh = 0; hh < 2; ++hh) {
                             const uint32_t a = op + hh * kLBO + (rho >> 3) * kSBO + (rho & 7) * 16;
-                            if (a % 16 || a + 16 > (uint32_t)kXBytes) return 30;
+                            if (a % 16 || a + 16 > (uint32_t)kXOpBytes) return 30;
                             if (used[a / 16]++) return 31;
                         }
                 }
@@ -1052,9 +1055,13 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
             return 33;
         for (int st = 0; st < kStages; ++st)
             if (stage_base(st) % 1024 || stage_d(st) + kDBytes > (uint32_t)kSmemBytes ||
-                stage_codes(st) + kCodesBytes != stage_x(st))
+                stage_codes(st) + kCodesBytes != stage_xraw(st) ||
+                stage_xraw(st) + kXRawBytes != stage_xop(st) || stage_xop(st) + kXOpBytes != stage_d(st))
                 return 34;
-        if (kSlots * kSlotCols > 512) return 35;
+        if (kTStages * kTStageCols > 512 || kS * kSlotCols != kTStageCols) return 35;
+        for (int r = 0; r < kM; ++r)
+            for (int c = 0; c < kS; ++c)
+                if (code_off(r, c) % 16 || code_off(r, c) + 16 > (uint32_t)kCodesBytes) return 36;
     }
     std::vector<std::vector<uint8_t>> cover(count);
     for (int i = 0; i < count; ++i)
@@ -1086,15 +1093,33 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
             cur_tile = s.tile;
             next_kb = s.kb0 + s.nblk;
             pos += s.nblk;
+            const int32_t w0 = window_of(s.kb0);
+            const int c0 = s.kb0 - w0;
+            if (w0 % kS || c0 + s.nblk > kS) return 7;  // inside one window
+            // TMA boxes: 16-byte aligned x, inside the row; first row inside
+            if ((16 * (int64_t)w0) % 16 || 16 * (int64_t)w0 >= sh[s.g].k / 2 ||
+                (int64_t)s.tile * kM >= sh[s.g].n)
+                return 11;
+            if (32 * (int64_t)w0 >= sh[s.g].k || (32 * (int64_t)w0 * 4) % 16) return 12;
+            if (G.d_box != (G.nb % 8 == 0 ? 1 : 0)) return 24;
+            if (G.d_box && ((2 * (int64_t)w0) % 16 || w0 >= G.nb || (G.nb * 2) % 16)) return 25;
+            if (!G.d_box) {
+                const int64_t dplane = round_up(sh[s.g].n * G.nb * 2, 16);
+                for (int r = 0; r < kM; ++r) {
+                    if ((int64_t)s.tile * kM + r >= sh[s.g].n) break;
+                    const DCopy dc = d_copy(G, s.tile, s.kb0, s.nblk, r);
+                    if (dc.src_off % 16 || dc.src_off < 0 || (dc.bytes != 16 && dc.bytes != 32) ||
+                        dc.src_off + dc.bytes > dplane || dc.lead + 2 * s.nblk > dc.bytes ||
+                        dc.bytes > (uint32_t)kDSlot)
+                        return 26;
+                }
+            }
             for (int i = 0; i < s.nblk; ++i) {
                 uint8_t& cv = cover[s.g][(size_t)s.tile * G.nb + s.kb0 + i];
                 if (cv) return 10;
                 cv = 1;
-                // TMA box: x aligned, inside the row; first row inside the matrix
-                const int64_t x = 16 * (int64_t)(s.kb0 + i);
-                if (x % 16 || x + 16 > sh[s.g].k / 2 || (int64_t)s.tile * kM >= sh[s.g].n) return 11;
-                // activation loads inside every token's row
-                if (32 * (int64_t)(s.kb0 + i) + 32 > sh[s.g].k) return 12;
+                // activation rows read by the x warps stay inside the raw box
+                if ((c0 + i) * 128 + 64 + 32 + 32 > kS * 128) return 12;
             }
             if (s.last) {
                 if (pos != hi && G.flat_begin + (int64_t)(s.tile + 1) * G.nb != pos) return 13;
@@ -1163,7 +1188,7 @@ int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks) {
             if (e < 0 || e > 31 || seen[e]++) ++bad;
         }
     }
-    std::vector<uint8_t> mem(kXBytes);
+    std::vector<uint8_t> mem(kXOpBytes);
     for (int64_t it = 0; it < blocks; ++it) {
         uint8_t codes[16];
         for (int j = 0; j < 16; ++j) codes[j] = (uint8_t)next();

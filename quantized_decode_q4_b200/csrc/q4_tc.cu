@@ -11,12 +11,16 @@
 // scale is applied exactly once, by the epilogue: y[t][r] += d[r][b] * D_b[r][t].
 //
 // Roles of the 14 warps of a CTA (one CTA per SM, persistent over a contiguous
-// range of (tile, block) units):
-//   producer (1 thread)   2-D TMA loads of the code bytes, 16 B x 128 rows per block
-//   x warps (4)           activations -> bf16 hi/lo B operands, scales -> binary32
+// range of (tile, block) units, walked in stages of up to 8 blocks):
+//   producer warp         per stage, on one barrier: the codes (one 2-D TMA box,
+//                         128-byte swizzle), the activations (one box, binary32)
+//                         and the scales (one box, or one bulk copy per row)
+//   x warps (4)           activations -> bf16 hi/lo B operands (shared -> shared)
 //   dequant warps (4)     codes -> (q - 8) bf16 A operands in tensor memory
-//   MMA thread (1)        tcgen05.mma M = 128, N = 16, K = 16 (2 or 4 per block)
-//   epilogue warps (4)    tcgen05.ld of each block's accumulator, scale, sum
+//   MMA thread (1)        tcgen05.mma M = 128, N = 16, K = 16, all blocks of a
+//                         stage chunk by chunk (consecutive MMAs accumulate into
+//                         different blocks), one commit per stage
+//   epilogue warps (4)    tcgen05.ld of the blocks' accumulators, scale, sum
 // Shared-memory stages and tensor-memory slots are handed over with mbarriers;
 // every wait is bounded and a wait that gives up records Q4_ERR_TIMEOUT, makes
 // every role leave its loop, and the kernel still waits for its own copies and
@@ -146,48 +150,101 @@ __device__ __forceinline__ bool warp_aborted(const Ctx& C) {
     return __shfl_sync(0xffffffffu, C.aborted() ? 1 : 0, 0) != 0;
 }
 
-// ---- producer: code bytes of every stage, one TMA box per block ----
-__device__ void run_producer(const Ctx& C, const q4t::Params& P) {
+// ---- producer warp: every TMA byte of a stage, on one barrier ----
+// Lane 0 issues the boxes (codes, activations, scales); with per-row scale
+// copies every lane issues the copies of rows lane, lane + 32, ... The
+// activations come from the previous kernel: the first kStages stages are
+// requested without them (weights only), then, after the wait on the previous
+// kernel, their activation boxes follow on the same barriers.
+template <int BT>
+__device__ void run_producer(const Ctx& C, const q4t::Params& P, int lane) {
+    constexpr uint32_t kXBox = (uint32_t)BT * q4t::kS * 32 * 4;
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
+    q4t::Walk wx = wk;
     q4t::Stage s;
     uint32_t q = 0;
-    while (!C.aborted() && wk.next(P, &s)) {
+    bool x_started = false;
+    while (!warp_aborted(C)) {
+        const bool has = wk.next(P, &s);
+        if (!x_started && (!has || q == (uint32_t)q4t::kStages)) {
+            pdl_wait();
+            if (lane == 0) {
+                for (uint32_t qq = 0; qq < q; ++qq) {
+                    q4t::Stage sx;
+                    wx.next(P, &sx);
+                    const int st = (int)(qq % q4t::kStages);
+                    tma_load_2d(C.sbase + q4t::stage_xraw(st), &P.maps[sx.g].x,
+                                32 * q4t::window_of(sx.kb0), 0, C.bar(q4t::kBarFull + st));
+                }
+            }
+            x_started = true;
+        }
+        if (!has) break;
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        // from the second round of stages on, the wait depends on roles that
-        // wait for the previous kernel: wait for it first, so that the bounded
-        // wait measures this kernel only
-        if (q == (uint32_t)q4t::kStages) pdl_wait();
-        if (!wait1(C, P, q4t::kBarStageEmpty + st, (v & 1u) ^ 1u)) break;
-        const uint32_t full = C.bar(q4t::kBarCodesFull + st);
-        mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarCodesFull + st)),
-                              (uint32_t)s.nblk * q4t::kBlockCodeBytes);
-        const uint32_t dst = C.sbase + q4t::stage_codes(st);
-        for (int i = 0; i < s.nblk; ++i)
-            tma_load_2d(dst + (uint32_t)i * q4t::kBlockCodeBytes, &P.tmap[s.g], 16 * (s.kb0 + i),
+        if (!waitw(C, P, q4t::kBarStageEmpty + st, (v & 1u) ^ 1u)) break;
+        const q4t::Desc& G = P.g[s.g];
+        const int32_t w0 = q4t::window_of(s.kb0);
+        const uint32_t full = C.bar(q4t::kBarFull + st);
+        uint32_t dbytes = 2048u;
+        q4t::DCopy dc[4];
+        if (!G.d_box) {
+            uint32_t mine = 0;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = lane + 32 * rr;
+                dc[rr] = q4t::d_copy(G, s.tile, s.kb0, s.nblk, r);
+                if ((int64_t)s.tile * q4t::kM + r < G.n) mine += dc[rr].bytes;
+            }
+            dbytes = __reduce_add_sync(0xffffffffu, mine);
+        }
+        if (lane == 0) {
+            mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarFull + st)),
+                                  (uint32_t)q4t::kCodesBytes + kXBox + dbytes);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            tma_load_2d(C.sbase + q4t::stage_codes(st), &P.maps[s.g].codes, 16 * w0,
                         s.tile * q4t::kM, full);
-        (void)full;
+            if (G.d_box)
+                tma_load_2d(C.sbase + q4t::stage_d(st), &P.maps[s.g].d, w0, s.tile * q4t::kM, full);
+            if (x_started)
+                tma_load_2d(C.sbase + q4t::stage_xraw(st), &P.maps[s.g].x, 32 * w0, 0, full);
+        }
+        if (!G.d_box) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = lane + 32 * rr;
+                if ((int64_t)s.tile * q4t::kM + r < G.n)
+                    bulk_g2s(C.smem + q4t::stage_d(st) + r * q4t::kDSlot,
+                             reinterpret_cast<const uint8_t*>(G.d) + dc[rr].src_off, dc[rr].bytes,
+                             reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarFull + st)));
+            }
+        }
         ++q;
     }
-    // every load issued lands before the kernel may exit: wait for the latest
+    // every copy issued lands before the kernel may exit: wait for the latest
     // phase of each stage that was filled
-    const uint32_t n = q < (uint32_t)q4t::kStages ? q : (uint32_t)q4t::kStages;
-    for (uint32_t k = 0; k < n; ++k) {
-        const uint32_t qq = q - 1 - k;
-        mbar_wait_bounded(
-            reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarCodesFull + (int)(qq % q4t::kStages))),
-            (qq / q4t::kStages) & 1u);
+    if (lane == 0) {
+        const uint32_t n = q < (uint32_t)q4t::kStages ? q : (uint32_t)q4t::kStages;
+        for (uint32_t k = 0; k < n; ++k) {
+            const uint32_t qq = q - 1 - k;
+            mbar_wait_bounded(
+                reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarFull + (int)(qq % q4t::kStages))),
+                (qq / q4t::kStages) & 1u);
+        }
     }
+    __syncwarp();
 }
 
-// ---- x warps: activations -> hi/lo B operands, scales -> binary32 ----
+// ---- x warps: activations (shared, binary32) -> hi/lo B operands ----
 template <int BT>
 __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
     constexpr bool kSplit = BT <= 8;
     constexpr int kMaxItems = (BT * q4t::kS * 4 + 127) / 128;
     const int tid = xw * 32 + lane;  // 0..127
-    pdl_wait();                      // activations may come from the previous kernel
+    pdl_wait();  // every stage barrier also waits for the activations
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
@@ -195,23 +252,12 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
     while (!warp_aborted(C) && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        if (!waitw(C, P, q4t::kBarStageEmpty + st, (v & 1u) ^ 1u)) break;
-        const q4t::Desc& G = P.g[s.g];
-        // loads first: scales of row tid, then this thread's activation rows
-        const int64_t row = (int64_t)s.tile * q4t::kM + tid;
-        uint16_t dv[q4t::kS];
-#pragma unroll
-        for (int i = 0; i < q4t::kS; ++i) dv[i] = 0;
-        if (row < G.n) {
-            const uint16_t* dr = G.d + row * G.nb + s.kb0;
-#pragma unroll
-            for (int i = 0; i < q4t::kS; ++i)
-                if (i < s.nblk) dv[i] = __ldg(dr + i);
-        }
+        if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;
+        const int c0 = s.kb0 - q4t::window_of(s.kb0);
         const int per_t = s.nblk * 4;
         const int items = P.b * per_t;
-        const int64_t k = (int64_t)G.nb * 32;
-        float4 xa[kMaxItems], xb[kMaxItems];
+        const uint8_t* raw = C.smem + q4t::stage_xraw(st);
+        uint8_t* xs = C.smem + q4t::stage_xop(st);
 #pragma unroll
         for (int m = 0; m < kMaxItems; ++m) {
             const int it = tid + 128 * m;
@@ -219,24 +265,9 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
                 const int t = it / per_t, rem = it - t * per_t;
                 const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
                 const float4* src = reinterpret_cast<const float4*>(
-                    G.x + t * k + 32 * (int64_t)(s.kb0 + i) + 16 * c2 + 8 * hh);
-                xa[m] = __ldg(src);
-                xb[m] = __ldg(src + 1);
-            }
-        }
-        float* dsm = reinterpret_cast<float*>(C.smem + q4t::stage_d(st));
-#pragma unroll
-        for (int i = 0; i < q4t::kS; ++i)
-            if (i < s.nblk) dsm[i * q4t::kM + tid] = __half2float(__ushort_as_half(dv[i]));
-        uint8_t* xs = C.smem + q4t::stage_x(st);
-#pragma unroll
-        for (int m = 0; m < kMaxItems; ++m) {
-            const int it = tid + 128 * m;
-            if (it < items) {
-                const int t = it / per_t, rem = it - t * per_t;
-                const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
-                const float e[8] = {xa[m].x, xa[m].y, xa[m].z, xa[m].w,
-                                    xb[m].x, xb[m].y, xb[m].z, xb[m].w};
+                    raw + t * (q4t::kS * 128) + (c0 + i) * 128 + c2 * 64 + hh * 32);
+                const float4 xa = src[0], xb = src[1];
+                const float e[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
                 uint4 H, L;
                 q4tm::split_row(e, &H, &L);
                 *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kSplit, i, c2, hh, t, 0)) = H;
@@ -246,7 +277,10 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
         // the MMA reads these operands through the async proxy
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(C.bar(q4t::kBarXFull + st));
+        if (lane == 0) {
+            mbar_arrive(C.bar(q4t::kBarXOpFull + st));
+            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
+        }
         ++q;
     }
 }
@@ -255,38 +289,33 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
 __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane) {
     const int r = dw * 32 + lane;
     const uint32_t tlane = C.tmem + ((uint32_t)(dw * 32) << 16);
+    pdl_wait();  // every stage barrier also waits for the activations
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0, j = 0;
+    uint32_t q = 0;
     while (!warp_aborted(C) && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        if (q == (uint32_t)(q4t::kSlots / q4t::kS)) pdl_wait();  // slots now wait for the epilogue
-        if (!waitw(C, P, q4t::kBarCodesFull + st, v & 1u)) break;
-        const uint8_t* codes = C.smem + q4t::stage_codes(st) + r * 16;
-        bool ok = true;
-        const uint32_t j0 = j;
+        const int ts = (int)(q & 1u);
+        const uint32_t u = q >> 1;
+        if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;
+        if (!waitw(C, P, q4t::kBarTEmpty + ts, (u & 1u) ^ 1u)) break;
+        tc_fence_after();
+        const uint8_t* codes = C.smem + q4t::stage_codes(st);
+        const int c0 = s.kb0 - q4t::window_of(s.kb0);
+        const uint32_t tcol = tlane + (uint32_t)(ts * q4t::kTStageCols);
         for (int i = 0; i < s.nblk; ++i) {
-            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
-            if (!waitw(C, P, q4t::kBarSlotEmpty + (int)p, (u & 1u) ^ 1u)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint4 qv = *reinterpret_cast<const uint4*>(codes + i * q4t::kBlockCodeBytes);
+            const uint4 qv = *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i));
             uint32_t a[16];
             q4tm::dequant_block(qv, a);
-            tc_st16(tlane + p * q4t::kSlotCols, a);
-            ++j;
+            tc_st16(tcol + (uint32_t)(i * q4t::kSlotCols), a);
         }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (!ok) break;
         if (lane == 0) {
-            for (uint32_t jj = j0; jj < j; ++jj)
-                mbar_arrive(C.bar(q4t::kBarAFull + (int)(jj % q4t::kSlots)));
+            mbar_arrive(C.bar(q4t::kBarAFull + ts));
             mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
         }
         ++q;
@@ -294,6 +323,8 @@ __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane
 }
 
 // ---- MMA thread ----
+// Per stage: for each chunk (and hi / lo part) the MMAs of all blocks in turn,
+// so that consecutive MMAs accumulate into different blocks' accumulators.
 template <int BT>
 __device__ void run_mma(const Ctx& C, const q4t::Params& P) {
     constexpr bool kSplit = BT <= 8;
@@ -301,39 +332,28 @@ __device__ void run_mma(const Ctx& C, const q4t::Params& P) {
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0, j = 0;
+    uint32_t q = 0;
     while (!C.aborted() && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        if (!wait1(C, P, q4t::kBarXFull + st, v & 1u)) break;
-        const uint32_t xs = C.sbase + q4t::stage_x(st);
-        bool ok = true;
-        for (int i = 0; i < s.nblk; ++i) {
-            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
-            if (!wait1(C, P, q4t::kBarAFull + (int)p, u & 1u)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t a = C.tmem + p * q4t::kSlotCols;
-            const uint32_t d = a + 16;
+        const int ts = (int)(q & 1u);
+        const uint32_t u = q >> 1;
+        if (!wait1(C, P, q4t::kBarXOpFull + st, v & 1u)) break;
+        if (!wait1(C, P, q4t::kBarAFull + ts, u & 1u)) break;
+        tc_fence_after();
+        const uint32_t xs = C.sbase + q4t::stage_xop(st);
+        const uint32_t t0 = C.tmem + (uint32_t)(ts * q4t::kTStageCols);
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                if (kSplit) {
-                    tc_mma(d, a + 8 * c2, q4t::smem_desc(xs + q4t::x_operand_off(true, i, c2, 0)),
-                           c2 != 0);
-                } else {
+        for (int c2 = 0; c2 < 2; ++c2)
 #pragma unroll
-                    for (int hl = 0; hl < 2; ++hl)
-                        tc_mma(d, a + 8 * c2,
-                               q4t::smem_desc(xs + q4t::x_operand_off(false, i, c2, hl)),
-                               (c2 | hl) != 0);
+            for (int hl = 0; hl < (kSplit ? 1 : 2); ++hl)
+                for (int i = 0; i < s.nblk; ++i) {
+                    const uint32_t a = t0 + (uint32_t)(i * q4t::kSlotCols);
+                    tc_mma(a + 16, a + 8 * c2,
+                           q4t::smem_desc(xs + q4t::x_operand_off(kSplit, i, c2, hl)),
+                           (c2 | hl) != 0);
                 }
-            }
-            tc_commit(C.bar(q4t::kBarDFull + (int)p));
-            ++j;
-        }
-        if (!ok) break;
+        tc_commit(C.bar(q4t::kBarDFull + ts));
         tc_commit(C.bar(q4t::kBarStageEmpty + st));
         ++q;
     }
@@ -385,53 +405,71 @@ __device__ __forceinline__ void finish_piece(const q4t::Params& P, const q4t::St
 }
 
 template <int BT>
-__device__ void run_epilogue(const Ctx& C, const q4t::Params& P, int ew, int lane) {
+__device__ __forceinline__ void accumulate(float (&acc)[BT], float dd, const uint32_t (&D)[16]) {
     constexpr bool kSplit = BT <= 8;
+#pragma unroll
+    for (int t = 0; t < BT; ++t) {
+        const float val = kSplit ? __uint_as_float(D[t]) + __uint_as_float(D[8 + t])
+                                 : __uint_as_float(D[t]);
+        acc[t] = fmaf(dd, val, acc[t]);
+    }
+}
+
+template <int BT>
+__device__ void run_epilogue(const Ctx& C, const q4t::Params& P, int ew, int lane) {
     const int r = ew * 32 + lane;
     const uint32_t tlane = C.tmem + ((uint32_t)(ew * 32) << 16);
     pdl_wait();  // partial sums, tickets and y are written below
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0, j = 0;
+    uint32_t q = 0;
     float acc[BT];
 #pragma unroll
     for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
     while (!warp_aborted(C) && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
+        const int ts = (int)(q & 1u);
+        const uint32_t u = q >> 1;
         if (s.first) {
 #pragma unroll
             for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
         }
-        if (!waitw(C, P, q4t::kBarXFull + st, v & 1u)) break;  // scales of the stage
-        const float* dsm = reinterpret_cast<const float*>(C.smem + q4t::stage_d(st)) + r;
-        bool ok = true;
-        for (int i = 0; i < s.nblk; ++i) {
-            const uint32_t p = j % q4t::kSlots, u = j / q4t::kSlots;
-            if (!waitw(C, P, q4t::kBarDFull + (int)p, u & 1u)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t D[16];
-            tc_ld16(tlane + p * q4t::kSlotCols + 16, D);
+        if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;  // the stage's scales
+        if (!waitw(C, P, q4t::kBarDFull + ts, u & 1u)) break;
+        tc_fence_after();
+        const q4t::Desc& G = P.g[s.g];
+        const int c0 = s.kb0 - q4t::window_of(s.kb0);
+        const bool live = (int64_t)s.tile * q4t::kM + r < G.n;
+        const uint8_t* dsm = C.smem + q4t::stage_d(st);
+        const uint16_t* drow =
+            G.d_box ? reinterpret_cast<const uint16_t*>(dsm + r * 16) + c0
+                    : reinterpret_cast<const uint16_t*>(
+                          dsm + r * q4t::kDSlot + q4t::d_copy(G, s.tile, s.kb0, s.nblk, r).lead);
+        const uint32_t tcol = tlane + (uint32_t)(ts * q4t::kTStageCols) + 16u;
+        for (int i0 = 0; i0 < s.nblk; i0 += 4) {
+            uint32_t D0[16], D1[16], D2[16], D3[16];
+            tc_ld16(tcol + (uint32_t)(i0 * q4t::kSlotCols), D0);
+            if (i0 + 1 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 1) * q4t::kSlotCols), D1);
+            if (i0 + 2 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 2) * q4t::kSlotCols), D2);
+            if (i0 + 3 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 3) * q4t::kSlotCols), D3);
             tc_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(C.bar(q4t::kBarSlotEmpty + (int)p));
-            const float dd = dsm[i * q4t::kM];
-#pragma unroll
-            for (int t = 0; t < BT; ++t) {
-                const float val = kSplit ? __uint_as_float(D[t]) + __uint_as_float(D[8 + t])
-                                         : __uint_as_float(D[t]);
-                acc[t] = fmaf(dd, val, acc[t]);
-            }
-            ++j;
+            const float d0 = live ? __half2float(__ushort_as_half(drow[i0])) : 0.0f;
+            accumulate<BT>(acc, d0, D0);
+            if (i0 + 1 < s.nblk)
+                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 1])) : 0.0f, D1);
+            if (i0 + 2 < s.nblk)
+                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 2])) : 0.0f, D2);
+            if (i0 + 3 < s.nblk)
+                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 3])) : 0.0f, D3);
         }
-        if (!ok) break;
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
+        if (lane == 0) {
+            mbar_arrive(C.bar(q4t::kBarTEmpty + ts));
+            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
+        }
         ++q;
         if (s.last) finish_piece<BT>(P, s, ew, lane, acc);
     }
@@ -452,23 +490,25 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
     if (threadIdx.x == 0) {
         uint64_t* b = reinterpret_cast<uint64_t*>(smem_raw);
         for (int st = 0; st < q4t::kStages; ++st) {
-            mbar_init(b + q4t::kBarCodesFull + st, 1);
-            mbar_init(b + q4t::kBarXFull + st, q4t::kArrivalsXFull);
+            mbar_init(b + q4t::kBarFull + st, 1);
+            mbar_init(b + q4t::kBarXOpFull + st, q4t::kArrivalsXOpFull);
             mbar_init(b + q4t::kBarStageEmpty + st, q4t::kArrivalsStageEmpty);
         }
-        for (int p = 0; p < q4t::kSlots; ++p) {
-            mbar_init(b + q4t::kBarAFull + p, q4t::kArrivalsAFull);
-            mbar_init(b + q4t::kBarDFull + p, 1);
-            mbar_init(b + q4t::kBarSlotEmpty + p, q4t::kArrivalsSlotEmpty);
+        for (int ts = 0; ts < q4t::kTStages; ++ts) {
+            mbar_init(b + q4t::kBarAFull + ts, q4t::kArrivalsAFull);
+            mbar_init(b + q4t::kBarDFull + ts, 1);
+            mbar_init(b + q4t::kBarTEmpty + ts, q4t::kArrivalsTEmpty);
         }
         mbar_init(b + q4t::kBarDone, 1);
-        *C.abort_flag = 0;
+        // the swizzled code box needs a 1024-byte aligned destination
+        *C.abort_flag = (C.sbase & 1023u) ? 1 : 0;
+        if (C.sbase & 1023u) atomicOr(P.ws, kTimeoutFlag);
         mbar_fence_init();
     }
     // operand rows of absent tokens stay zero for the whole launch
     for (int st = 0; st < q4t::kStages; ++st)
-        for (int off = threadIdx.x * 16; off < q4t::kXBytes; off += q4t::kThreads * 16)
-            *reinterpret_cast<uint4*>(smem_raw + q4t::stage_x(st) + off) = make_uint4(0, 0, 0, 0);
+        for (int off = threadIdx.x * 16; off < q4t::kXOpBytes; off += q4t::kThreads * 16)
+            *reinterpret_cast<uint4*>(smem_raw + q4t::stage_xop(st) + off) = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (warp == 0) {
         tc_alloc(C.sbase + q4t::kTmemAddrOff, q4t::kTmemCols);
@@ -488,8 +528,7 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
     } else if (warp < q4t::kProdWarp) {
         run_x<BT>(C, P, warp - q4t::kXWarp0, lane);
     } else if (warp == q4t::kProdWarp) {
-        if (lane == 0) run_producer(C, P);
-        __syncwarp();
+        run_producer<BT>(C, P, lane);
     } else {
         if (lane == 0) run_mma<BT>(C, P);
         __syncwarp();
@@ -556,24 +595,50 @@ cudaError_t launch_one(const q4t::Params& P, bool pdl, cudaStream_t stream) {
 
 }  // namespace
 
-// Tensor map of the code plane of an n x k matrix: uint8 [n][k/2], box of
-// 16 bytes (one block) x 128 rows, no swizzle; rows past n read as zero.
-cudaError_t encode_code_map(CUtensorMap* map, const uint8_t* qs, int64_t n, int64_t k) {
+// Token count a launch is compiled for: the smallest of 2, 4, 8, 16 >= b.
+int tc_tokens(int b) { return b <= 2 ? 2 : b <= 4 ? 4 : b <= 8 ? 8 : 16; }
+
+namespace {
+cudaError_t encode(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n};
-    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
-    const cuuint32_t box[2] = {16u, (cuuint32_t)q4t::kM};
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(qs), dims,
-                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
+}  // namespace
 
-// Token count a launch is compiled for: the smallest of 2, 4, 8, 16 >= b.
-int tc_tokens(int b) { return b <= 2 ? 2 : b <= 4 ? 4 : b <= 8 ? 8 : 16; }
+// Tensor maps of one GEMV for b tokens (rows and columns past the ends read as
+// zero): code plane uint8 [n][k/2], box 128 B x 128 rows with the 128-byte
+// swizzle; activations binary32 [b][k], box 256 x (b rounded up to the compiled
+// token count); scale plane uint16 [n][k/32], box 8 x 128 rows, when its row
+// stride is a multiple of 16 bytes (*d_box = 1).
+cudaError_t encode_tc_maps(q4t::Maps* maps, int32_t* d_box, const uint8_t* qs, const uint16_t* d,
+                           const float* x, int64_t n, int64_t k, int b) {
+    cudaError_t e = encode(&maps->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, qs, (uint64_t)(k / 2),
+                           (uint64_t)n, (uint64_t)(k / 2), 128u, (uint32_t)q4t::kM,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = encode(&maps->x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, (uint64_t)k, (uint64_t)b,
+               (uint64_t)(k * 4), (uint32_t)(q4t::kS * 32), (uint32_t)tc_tokens(b),
+               CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    const int64_t nb = k / 32;
+    *d_box = nb % 8 == 0 ? 1 : 0;
+    if (*d_box)
+        e = encode(&maps->d, CU_TENSOR_MAP_DATA_TYPE_UINT16, d, (uint64_t)nb, (uint64_t)n,
+                   (uint64_t)(nb * 2), (uint32_t)q4t::kS, (uint32_t)q4t::kM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    return e;
+}
+
 
 cudaError_t setup_tc_kernels(int optin_smem) {
     cudaError_t e;

@@ -6,21 +6,32 @@
 // work is one K block (32 weights) of one M tile (128 rows) of one GEMV. Units
 // are ordered (GEMV, tile, block) and laid end to end in one "flat" space of F
 // units; CTA c of G owns units [F c / G, F (c + 1) / G). The part of a CTA's
-// range inside one tile is a piece; a piece is walked in stages of up to kS
-// blocks. A tile covered by several pieces (several CTAs) is finished by the
-// last one to arrive: each piece stores its 128 x b partial sums in its own
-// slot (slot = CTA index - first CTA of the tile), and the last arriver adds
-// the slots in order (deterministic).
+// range inside one tile is a piece; a piece is walked in stages that never
+// cross a multiple of kS blocks, so that every stage lies inside one aligned
+// group of kS blocks (the "window" [w0, w0 + kS), w0 = kb0 - kb0 % kS) and
+// every TMA box of a stage starts at a 16-byte aligned coordinate. A tile
+// covered by several pieces (several CTAs) is finished by the last one to
+// arrive: each piece stores its 128 x b partial sums in its own slot (slot =
+// CTA index - first CTA of the tile), and the last arriver adds the slots in
+// order (deterministic).
 //
-// Per stage, shared memory holds the code bytes of the stage's blocks (block i
-// at codes + 2048 i, row r at + 16 r: one 2-D TMA box of 16 bytes x 128 rows per
-// block), the activations as the MMA's B operand (bf16 hi and lo parts, in the
-// canonical K-major layout without swizzle: 8 x 16-byte core matrices) and the
-// blocks' scales as binary32 (d[i][r]).
+// Per stage, shared memory holds:
+//   codes   the window's code bytes, one TMA box of 128 B x 128 rows with the
+//           128-byte swizzle: block c of the window, row r at
+//           r * 128 + ((c ^ (r % 8)) * 16)
+//   xraw    the window's activations, one TMA box of 256 binary32 x 16 tokens
+//           (token t at t * 1024 bytes; absent tokens read as zero)
+//   xop     the stage's activations as the MMA's B operand: bf16 hi and lo parts
+//           in the canonical K-major layout without swizzle (8 x 16-byte core
+//           matrices), written by the x warps from xraw
+//   d       the window's binary16 scales: one TMA box of 8 x 128 rows
+//           ([r][8]) when the row stride of the scale plane is a multiple of 16
+//           bytes, else one 16-byte aligned bulk copy per row into a 32-byte
+//           slot per row (the stage's scales at an offset inside it)
 //
-// Tensor memory (512 columns x 128 lanes) holds kSlots slots of 32 columns, one
-// per block in flight: columns [0, 16) are the A operand (row r = lane r, the
-// block's 32 values of (q - 8) as bf16 pairs), columns [16, 32) the block's
+// Tensor memory (512 columns x 128 lanes) holds two tensor stages of kS blocks;
+// block i of tensor stage ts uses columns ts * 256 + 32 i: [0, 16) the A operand
+// (row r = lane r, the block's 32 values (q - 8) as bf16 pairs), [16, 32) its
 // accumulator D (128 x 16, binary32).
 #pragma once
 
@@ -37,69 +48,67 @@
 
 namespace q4t {
 
-#ifndef Q4_TC_STAGES
-#define Q4_TC_STAGES 5
-#endif
-#ifndef Q4_TC_STAGE_BLOCKS
-#define Q4_TC_STAGE_BLOCKS 8
-#endif
-
-constexpr int kM = 128;                 // rows per tile (MMA M)
-constexpr int kN = 16;                  // MMA N
-constexpr int kS = Q4_TC_STAGE_BLOCKS;  // K blocks per stage
-constexpr int kStages = Q4_TC_STAGES;   // shared-memory ring depth
-constexpr int kSlots = 16;              // tensor-memory slots
-constexpr int kSlotCols = 32;
-constexpr int kTmemCols = kSlots * kSlotCols;  // 512
-constexpr int kBlockCodeBytes = kM * 16;       // 2048
-constexpr int kBlockXBytes = 2048;             // 2 chunks x (hi, lo) x 512 B
-constexpr int kCodesBytes = kS * kBlockCodeBytes;
-constexpr int kXBytes = kS * kBlockXBytes;
-constexpr int kDBytes = kS * kM * 4;
-constexpr int kStageBytes = kCodesBytes + kXBytes + kDBytes;
-constexpr int kHeaderBytes = 1024;  // barriers, tensor-memory address, ticket broadcast
+constexpr int kM = 128;        // rows per tile (MMA M)
+constexpr int kN = 16;         // MMA N
+constexpr int kS = 8;          // K blocks per window (and at most per stage)
+constexpr int kStages = 4;     // shared-memory ring depth
+constexpr int kTStages = 2;    // tensor-memory stages
+constexpr int kSlotCols = 32;  // tensor-memory columns per block
+constexpr int kTStageCols = kS * kSlotCols;     // 256
+constexpr int kTmemCols = kTStages * kTStageCols;  // 512
+constexpr int kMaxTokens = 16;
+constexpr int kCodesBytes = kM * 128;               // 16 KB
+constexpr int kXRawBytes = kMaxTokens * kS * 32 * 4;  // 16 KB
+constexpr int kBlockXBytes = 2048;                  // 2 chunks x (hi, lo) x 512 B
+constexpr int kXOpBytes = kS * kBlockXBytes;        // 16 KB
+constexpr int kDSlot = 32;                          // bytes per row (per-row copies)
+constexpr int kDBytes = kM * kDSlot;                // 4 KB
+constexpr int kStageBytes = kCodesBytes + kXRawBytes + kXOpBytes + kDBytes;
+constexpr int kHeaderBytes = 1024;  // barriers, tensor-memory address, abort flag
 constexpr int kSmemBytes = kHeaderBytes + kStages * kStageBytes;
 
 // warp roles
 constexpr int kDequantWarp0 = 0;  // 4 warps: codes -> (q - 8) bf16 into tensor memory
 constexpr int kEpiWarp0 = 4;      // 4 warps: accumulators x scale, partial sums, y
-constexpr int kXWarp0 = 8;        // 4 warps: activations -> bf16 hi/lo, scales -> binary32
-constexpr int kProdWarp = 12;     // 1 thread: TMA loads of the code bytes
+constexpr int kXWarp0 = 8;        // 4 warps: xraw -> bf16 hi/lo B operands
+constexpr int kProdWarp = 12;     // TMA loads (lane 0) and per-row scale copies (all lanes)
 constexpr int kMmaWarp = 13;      // 1 thread: tcgen05.mma issue
 constexpr int kWarps = 14;
 constexpr int kThreads = kWarps * 32;
 
-static_assert(kS >= 1 && kS <= kSlots, "stage size");
-static_assert(kStageBytes % 1024 == 0, "stage alignment");
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled box");
 
 // barrier indices (uint64 words at the start of shared memory)
-constexpr int kBarCodesFull = 0;                       // [kStages]
-constexpr int kBarXFull = kBarCodesFull + kStages;     // [kStages]
-constexpr int kBarStageEmpty = kBarXFull + kStages;    // [kStages]
-constexpr int kBarAFull = kBarStageEmpty + kStages;    // [kSlots]
-constexpr int kBarDFull = kBarAFull + kSlots;          // [kSlots]
-constexpr int kBarSlotEmpty = kBarDFull + kSlots;      // [kSlots]
-constexpr int kBarDone = kBarSlotEmpty + kSlots;       // 1
+constexpr int kBarFull = 0;                          // [kStages] every TMA byte of the stage
+constexpr int kBarXOpFull = kBarFull + kStages;      // [kStages] B operands written
+constexpr int kBarStageEmpty = kBarXOpFull + kStages;  // [kStages]
+constexpr int kBarAFull = kBarStageEmpty + kStages;  // [kTStages]
+constexpr int kBarDFull = kBarAFull + kTStages;      // [kTStages]
+constexpr int kBarTEmpty = kBarDFull + kTStages;     // [kTStages]
+constexpr int kBarDone = kBarTEmpty + kTStages;      // 1
 constexpr int kNumBars = kBarDone + 1;
-constexpr int kTmemAddrOff = 8 * kNumBars;            // uint32 written by tcgen05.alloc
-constexpr int kTicketOff = kTmemAddrOff + 4;          // uint32 ticket broadcast
-constexpr int kAbortOff = kTicketOff + 4;             // int32 abort flag
+constexpr int kTmemAddrOff = 8 * kNumBars;  // uint32 written by tcgen05.alloc
+constexpr int kAbortOff = kTmemAddrOff + 4;  // int32 abort flag
 static_assert(kAbortOff + 4 <= kHeaderBytes, "header");
 
 // arrivals per barrier phase
-constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 1;  // dequant warps, epilogue warps, MMA commit
-constexpr uint32_t kArrivalsXFull = 4;               // x warps
-constexpr uint32_t kArrivalsAFull = 4;               // dequant warps
-constexpr uint32_t kArrivalsSlotEmpty = 4;           // epilogue warps
+constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 4 + 1;  // dequant, x, epilogue warps; MMA commit
+constexpr uint32_t kArrivalsXOpFull = 4;
+constexpr uint32_t kArrivalsAFull = 4;
+constexpr uint32_t kArrivalsTEmpty = 4;
 
 Q4T_HD uint32_t stage_base(int st) { return (uint32_t)(kHeaderBytes + st * kStageBytes); }
 Q4T_HD uint32_t stage_codes(int st) { return stage_base(st); }
-Q4T_HD uint32_t stage_x(int st) { return stage_base(st) + kCodesBytes; }
-Q4T_HD uint32_t stage_d(int st) { return stage_base(st) + kCodesBytes + kXBytes; }
+Q4T_HD uint32_t stage_xraw(int st) { return stage_base(st) + kCodesBytes; }
+Q4T_HD uint32_t stage_xop(int st) { return stage_base(st) + kCodesBytes + kXRawBytes; }
+Q4T_HD uint32_t stage_d(int st) { return stage_base(st) + kCodesBytes + kXRawBytes + kXOpBytes; }
 
-// Byte offset, inside a stage's activation region, of the 16-byte row holding
-// MMA positions [8 hh, 8 hh + 8) of chunk c2 (16 K values) of block i for MMA
-// row `row` (0..15) of operand part `hl` (0 = hi, 1 = lo). With at most 8
+// Code bytes of block c (0..kS-1) of the window, row r, inside the swizzled box.
+Q4T_HD uint32_t code_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// Byte offset, inside a stage's operand region, of the 16-byte row holding MMA
+// positions [8 hh, 8 hh + 8) of chunk c2 (16 K values) of stage block i for
+// MMA row `row` (0..15) of operand part `hl` (0 = hi, 1 = lo). With at most 8
 // tokens (split) the hi parts of tokens t are rows t and the lo parts rows
 // 8 + t of one 16-row operand (1 KB per block); with more tokens the hi and lo
 // parts are two 16-row operands (2 KB per block) accumulated into the same D.
@@ -108,8 +117,7 @@ Q4T_HD uint32_t stage_d(int st) { return stage_base(st) + kCodesBytes + kXBytes;
 constexpr uint32_t kLBO = 256;  // between the two K halves of an operand
 constexpr uint32_t kSBO = 128;  // between the two 8-row groups
 Q4T_HD uint32_t x_operand_off(bool split, int i, int c2, int hl) {
-    return split ? (uint32_t)(i * 1024 + c2 * 512)
-                 : (uint32_t)(i * 2048 + c2 * 1024 + hl * 512);
+    return split ? (uint32_t)(i * 1024 + c2 * 512) : (uint32_t)(i * 2048 + c2 * 1024 + hl * 512);
 }
 Q4T_HD uint32_t x_row_off(bool split, int i, int c2, int hh, int t, int hl) {
     const int row = split ? (hl ? 8 + t : t) : t;
@@ -153,18 +161,25 @@ struct Desc {
     int32_t tiles;       // ceil(n / 128)
     int64_t flat_begin;  // first unit of this GEMV in the flat space
     int64_t part_off;    // floats: partial sums [tiles][maxp][b][128]
-    int64_t ticket_off;  // uint32: one ticket per tile
+    int64_t ticket_off;  // uint32: four tickets per tile (one per epilogue warp)
     int32_t maxp;        // partial slots per tile (1: no split tiles)
-    int32_t pad_;
+    int32_t d_box;       // 1: scales by one TMA box per stage (nb % 8 == 0)
+};
+
+// Tensor maps of GEMV g: codes uint8 [n][k/2] (box 128 x 128, 128-byte swizzle),
+// activations binary32 [b][k] (box 256 x 16), scales uint16 [n][nb] (box 8 x 128,
+// only when d_box).
+struct Maps {
+    CUtensorMap codes, x, d;
 };
 
 struct Params {
-    CUtensorMap tmap[Q4_MAX_GROUP];  // code bytes of GEMV g: uint8 [n][k/2], box 16 x 128
+    Maps maps[Q4_MAX_GROUP];
     Desc g[Q4_MAX_GROUP];
     int32_t count;
-    int32_t b;        // tokens
-    int64_t total;    // F, < 2^31
-    int32_t grid;     // G
+    int32_t b;      // tokens
+    int64_t total;  // F, < 2^31
+    int32_t grid;   // G
     int32_t pad_;
     uint32_t* ws;
 };
@@ -182,10 +197,12 @@ struct Stage {
     int g;
     int32_t tile;
     int32_t kb0;    // first block
-    int32_t nblk;   // blocks (1..kS)
+    int32_t nblk;   // blocks (1..kS), all inside the window of kb0
     bool first;     // first stage of a piece
     bool last;      // last stage of a piece
 };
+
+Q4T_HD int32_t window_of(int32_t kb0) { return kb0 - kb0 % kS; }
 
 struct Walk {
     int64_t pos, hi;
@@ -209,10 +226,11 @@ struct Walk {
         const int64_t tile_end = G.flat_begin + (int64_t)(tile + 1) * nb;
         const int64_t pend = tile_end < hi ? tile_end : hi;
         const int64_t left = pend - pos;
+        const int32_t room = kS - kb % kS;
         s->g = g;
         s->tile = (int32_t)tile;
         s->kb0 = kb;
-        s->nblk = (int32_t)(left < kS ? left : kS);
+        s->nblk = (int32_t)(left < room ? left : room);
         s->first = fresh;
         s->last = pos + s->nblk == pend;
         pos += s->nblk;
@@ -228,6 +246,24 @@ Q4T_HD void tile_pieces(const Params& P, const Desc& G, int32_t tile, int c, int
     const int c0 = owner(f0, P.total, P.grid), c1 = owner(f1, P.total, P.grid);
     *np = c1 - c0 + 1;
     *slot = c - c0;
+}
+
+// Per-row scale copy of row r of a stage (when the scales are not one box):
+// the 16-byte aligned superset of the stage's scales, and where the scale of
+// stage block i lands: slot r, byte (src_off % 16) + 2 i.
+struct DCopy {
+    int64_t src_off;  // byte offset in the scale plane (16-byte aligned)
+    uint32_t bytes;   // 16 or 32
+    uint32_t lead;    // (first scale's byte offset) % 16
+};
+Q4T_HD DCopy d_copy(const Desc& G, int32_t tile, int32_t kb0, int32_t nblk, int r) {
+    const int64_t a = (((int64_t)tile * kM + r) * G.nb + kb0) * 2;
+    const int64_t a0 = a & ~(int64_t)15;
+    DCopy c;
+    c.src_off = a0;
+    c.lead = (uint32_t)(a - a0);
+    c.bytes = (uint32_t)(((a + 2 * nblk + 15) & ~(int64_t)15) - a0);
+    return c;
 }
 
 }  // namespace q4t
