@@ -1022,43 +1022,68 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {
     if (plan_tc(sh, count, b, base, &P, &tickets, &end) != Q4_OK) return 2;
     if (kSmemBytes > (int)kMaxSmem || 2 * kSmemBytes <= 228 * 1024) return 3;  // one CTA per SM
     if (P.grid < 1 || P.grid > kNumSMs || P.grid > P.total) return 4;
-    const bool split = q4k::tc_tokens(b) <= 8;
+    const int bt = q4k::tc_tokens(b);
+    const int nn = mma_n(bt);
     // operand layout: every (block, chunk, K half, MMA row) has its own 16-byte
-    // row inside the stage's activation region, and the MMA descriptor of each
-    // operand addresses exactly those rows
+    // row inside the stage's activation region, the MMA descriptor of each
+    // operand addresses exactly those rows, and every token's hi and lo rows
+    // are the operand's rows t and N / 2 + t
     {
         std::vector<int> used(kXOpBytes / 16, 0);
         for (int i = 0; i < kS; ++i)
-            for (int c2 = 0; c2 < 2; ++c2)
-                for (int hl = 0; hl < (split ? 1 : 2); ++hl) {
-                    const uint32_t op = x_operand_off(split, i, c2, hl);
-                    for (int rho = 0; rho < kN; ++rho)
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t a = op + hh * kLBO + (rho >> 3) * kSBO + (rho & 7) * 16;
-                            if (a % 16 || a + 16 > (uint32_t)kXOpBytes) return 30;
-                            if (used[a / 16]++) return 31;
-                        }
-                }
-        for (int i = 0; i < kS; ++i)
-            for (int c2 = 0; c2 < 2; ++c2)
-                for (int t = 0; t < (split ? 8 : 16); ++t)
+            for (int c2 = 0; c2 < 2; ++c2) {
+                const uint32_t op = x_operand_off(nn, i, c2);
+                for (int rho = 0; rho < nn; ++rho)
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t a = op + hh * lbo(nn) + (rho >> 3) * kSBO + (rho & 7) * 16;
+                        if (a % 16 || a + 16 > (uint32_t)kXOpBytes) return 30;
+                        if (used[a / 16]++) return 31;
+                    }
+                for (int t = 0; t < bt; ++t)
                     for (int hh = 0; hh < 2; ++hh)
                         for (int hl = 0; hl < 2; ++hl) {
-                            const int rho = split ? (hl ? 8 + t : t) : t;
-                            const uint32_t want = x_operand_off(split, i, c2, hl) + hh * kLBO +
-                                                  (rho >> 3) * kSBO + (rho & 7) * 16;
-                            if (x_row_off(split, i, c2, hh, t, hl) != want) return 32;
+                            const int rho = hl ? nn / 2 + t : t;
+                            const uint32_t want =
+                                op + hh * lbo(nn) + (rho >> 3) * kSBO + (rho & 7) * 16;
+                            if (x_row_off(nn, i, c2, hh, t, hl) != want) return 32;
                         }
-        const uint64_t dsc = smem_desc(0x1230u);
-        if ((dsc & 0x3FFF) != (0x1230u >> 4) || ((dsc >> 16) & 0x3FFF) != kLBO / 16 ||
+            }
+        if (bt > nn / 2) return 32;
+        const uint64_t dsc = smem_desc(0x1230u, nn);
+        if ((dsc & 0x3FFF) != (0x1230u >> 4) || ((dsc >> 16) & 0x3FFF) != lbo(nn) / 16 ||
             ((dsc >> 32) & 0x3FFF) != kSBO / 16 || ((dsc >> 46) & 3) != 1 || (dsc >> 61) != 0)
+            return 33;
+        // descriptors advance by adding (offset >> 4) to the 14-bit start address
+        if ((kSmemBytes >> 4) >= (1 << 14)) return 33;
+        for (int i = 0; i < kS; ++i)
+            for (int c2 = 0; c2 < 2; ++c2)
+                if (smem_desc(0x400u, nn) + (uint64_t)((2 * i + c2) * nn * 32 >> 4) !=
+                    smem_desc(0x400u + x_operand_off(nn, i, c2), nn))
+                    return 33;
+        const uint32_t id = instr_desc(nn);
+        if (((id >> 17) & 63) != (uint32_t)nn / 8 || ((id >> 24) & 31) != 8 || ((id >> 4) & 3) != 1 ||
+            ((id >> 7) & 7) != 1 || ((id >> 10) & 7) != 1)
             return 33;
         for (int st = 0; st < kStages; ++st)
             if (stage_base(st) % 1024 || stage_d(st) + kDBytes > (uint32_t)kSmemBytes ||
                 stage_codes(st) + kCodesBytes != stage_xraw(st) ||
                 stage_xraw(st) + kXRawBytes != stage_xop(st) || stage_xop(st) + kXOpBytes != stage_d(st))
                 return 34;
-        if (kTStages * kTStageCols > 512 || kS * kSlotCols != kTStageCols) return 35;
+        // tensor memory: the A ring and the D ring are disjoint and inside 512 columns
+        std::vector<int> cols(kTmemCols, 0);
+        for (int sa = 0; sa < kRingA; ++sa)
+            for (int i = 0; i < kQ; ++i)
+                for (int c = 0; c < kACols; ++c) {
+                    const uint32_t col = a_col(sa, i) + c;
+                    if (col >= (uint32_t)kTmemCols || cols[col]++) return 35;
+                }
+        if (ring_d(bt) > kMaxRingD || ring_d(bt) < 2) return 35;
+        for (int sd = 0; sd < ring_d(bt); ++sd)
+            for (int i = 0; i < kQ; ++i)
+                for (int c = 0; c < nn; ++c) {
+                    const uint32_t col = d_col(bt, sd, i) + c;
+                    if (col >= (uint32_t)kTmemCols || cols[col]++) return 35;
+                }
         for (int r = 0; r < kM; ++r)
             for (int c = 0; c < kS; ++c)
                 if (code_off(r, c) % 16 || code_off(r, c) + 16 > (uint32_t)kCodesBytes) return 36;
@@ -1216,27 +1241,29 @@ int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks) {
             if (aval[kap] != (double)(q[element_at(kap)] - 8)) ++bad;
         }
         for (int mode = 0; mode < 2; ++mode) {
-            const bool split = mode == 0;
+            const int nn = mode == 0 ? 16 : 32;
+            const int t = mode == 0 ? 5 : 13;  // a token of each layout
             std::fill(mem.begin(), mem.end(), 0);
-            // token 0 of block 0 in the layout the x warps write
+            // token t of block 0 in the layout the x warps write
             for (int c2 = 0; c2 < 2; ++c2)
                 for (int hh = 0; hh < 2; ++hh) {
                     float e[8];
                     for (int m = 0; m < 8; ++m) e[m] = x[16 * c2 + 8 * hh + m];
                     uint4 H, L;
                     q4tm::split_row(e, &H, &L);
-                    std::memcpy(&mem[x_row_off(split, 0, c2, hh, 0, 0)], &H, 16);
-                    std::memcpy(&mem[x_row_off(split, 0, c2, hh, 0, 1)], &L, 16);
+                    std::memcpy(&mem[x_row_off(nn, 0, c2, hh, t, 0)], &H, 16);
+                    std::memcpy(&mem[x_row_off(nn, 0, c2, hh, t, 1)], &L, 16);
                 }
-            // the MMA: D[row 0][col] = sum_kappa A[kappa] B[col][kappa] over both chunks
+            // the MMA: D[row 0][col] = sum_kappa A[kappa] B[col][kappa] over both
+            // chunks, at the addresses the descriptor gives; the epilogue adds
+            // columns t (hi) and N / 2 + t (lo)
             double dsum = 0.0;
             for (int hl = 0; hl < 2; ++hl) {
-                const int col = split ? (hl ? 8 : 0) : 0;
+                const int col = hl ? nn / 2 + t : t;
                 for (int kap = 0; kap < 32; ++kap) {
                     const int c2 = kap >> 4, kk = kap & 15;
-                    const uint32_t op = x_operand_off(split, 0, c2, split ? 0 : hl);
-                    const uint32_t addr = op + (kk >> 3) * kLBO + (col >> 3) * kSBO + (col & 7) * 16 +
-                                          (kk & 7) * 2;
+                    const uint32_t addr = x_operand_off(nn, 0, c2) + (kk >> 3) * lbo(nn) +
+                                          (col >> 3) * kSBO + (col & 7) * 16 + (kk & 7) * 2;
                     uint16_t bits;
                     std::memcpy(&bits, &mem[addr], 2);
                     dsum += aval[kap] * (double)q4tm::bf16_value(bits);

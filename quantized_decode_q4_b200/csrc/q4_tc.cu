@@ -5,23 +5,33 @@
 // weights are dequantised into fast on-chip memory and reused there. Here the
 // on-chip memory is tensor memory: each 32-weight block of a 128-row tile is
 // dequantised once to (q - 8) as bf16 (exact) and written with tcgen05.st into
-// a tensor-memory slot, and tcgen05.mma multiplies it with the tokens'
-// activations held in shared memory as bf16 hi + lo parts (x = hi + lo to
-// 2^-16 relative). Every block has its own binary32 accumulator, so its binary16
-// scale is applied exactly once, by the epilogue: y[t][r] += d[r][b] * D_b[r][t].
+// tensor memory, and tcgen05.mma multiplies it with the tokens' activations held
+// in shared memory as bf16 hi + lo parts (x = hi + lo to 2^-16 relative; both
+// parts are columns of one N = 16 or 32 operand). Every block has its own
+// binary32 accumulator, so its binary16 scale is applied exactly once, by the
+// epilogue: y[t][r] += d[r][b] * (D_b[r][t] + D_b[r][N/2 + t]).
 //
-// Roles of the 14 warps of a CTA (one CTA per SM, persistent over a contiguous
+// Measured on B200 (M = 128, K = 16, bf16): one thread issues an MMA about
+// every 50 cycles for any N up to 64; two issuing threads reach about 25; an
+// N = 256 MMA takes 128 cycles (the tensor core's peak). With N = 16 or 32 the
+// tensor core is bound by issue, so two threads issue alternate quads; the
+// dequant fills the A ring quad by quad (4 blocks) as soon as a quad's earlier
+// MMAs are done, and the accumulators live in a separate D ring read by the
+// epilogue.
+//
+// Roles of the 15 warps of a CTA (one CTA per SM, persistent over a contiguous
 // range of (tile, block) units, walked in stages of up to 8 blocks):
 //   producer warp         per stage, on one barrier: the codes (one 2-D TMA box,
 //                         128-byte swizzle), the activations (one box, binary32)
 //                         and the scales (one box, or one bulk copy per row)
 //   x warps (4)           activations -> bf16 hi/lo B operands (shared -> shared)
 //   dequant warps (4)     codes -> (q - 8) bf16 A operands in tensor memory
-//   MMA thread (1)        tcgen05.mma M = 128, N = 16, K = 16, all blocks of a
-//                         stage chunk by chunk (consecutive MMAs accumulate into
-//                         different blocks), one commit per stage
+//   MMA issuers (2)       tcgen05.mma M = 128, N = 16 or 32, K = 16, one thread
+//                         each, quads alternating; per quad all blocks chunk by
+//                         chunk (consecutive MMAs accumulate into different
+//                         blocks), two commits per quad
 //   epilogue warps (4)    tcgen05.ld of the blocks' accumulators, scale, sum
-// Shared-memory stages and tensor-memory slots are handed over with mbarriers;
+// Shared-memory stages and tensor-memory quads are handed over with mbarriers;
 // every wait is bounded and a wait that gives up records Q4_ERR_TIMEOUT, makes
 // every role leave its loop, and the kernel still waits for its own copies and
 // MMAs before it frees tensor memory and returns.
@@ -77,14 +87,14 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                      bar)
                  : "memory");
 }
-// D[128 x 16] (+)= A[128 x 16] (tensor memory) * B[16 x 16]^T (shared memory)
+// D[128 x N] (+)= A[128 x 16] (tensor memory) * B[N x 16]^T (shared memory)
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t accumulate) {
+                                       uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, {%5, %5, %5, %5}, p;\n}\n" ::"r"(
             d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(q4t::kInstrDesc), "r"(0u)
+        "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(idesc), "r"(0u)
         : "memory");
 }
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
@@ -241,7 +251,7 @@ __device__ void run_producer(const Ctx& C, const q4t::Params& P, int lane) {
 // ---- x warps: activations (shared, binary32) -> hi/lo B operands ----
 template <int BT>
 __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
-    constexpr bool kSplit = BT <= 8;
+    constexpr int kN = q4t::mma_n(BT);
     constexpr int kMaxItems = (BT * q4t::kS * 4 + 127) / 128;
     const int tid = xw * 32 + lane;  // 0..127
     pdl_wait();  // every stage barrier also waits for the activations
@@ -270,8 +280,8 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
                 const float e[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
                 uint4 H, L;
                 q4tm::split_row(e, &H, &L);
-                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kSplit, i, c2, hh, t, 0)) = H;
-                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kSplit, i, c2, hh, t, 1)) = L;
+                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 0)) = H;
+                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 1)) = L;
             }
         }
         // the MMA reads these operands through the async proxy
@@ -285,7 +295,7 @@ __device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
     }
 }
 
-// ---- dequant warps: codes -> (q - 8) bf16 in tensor memory ----
+// ---- dequant warps: codes -> (q - 8) bf16 in tensor memory, quad by quad ----
 __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane) {
     const int r = dw * 32 + lane;
     const uint32_t tlane = C.tmem + ((uint32_t)(dw * 32) << 16);
@@ -293,68 +303,103 @@ __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0;
-    while (!warp_aborted(C) && wk.next(P, &s)) {
+    uint32_t q = 0, j = 0;
+    bool ok = true;
+    while (ok && !warp_aborted(C) && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        const int ts = (int)(q & 1u);
-        const uint32_t u = q >> 1;
         if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;
-        if (!waitw(C, P, q4t::kBarTEmpty + ts, (u & 1u) ^ 1u)) break;
-        tc_fence_after();
         const uint8_t* codes = C.smem + q4t::stage_codes(st);
         const int c0 = s.kb0 - q4t::window_of(s.kb0);
-        const uint32_t tcol = tlane + (uint32_t)(ts * q4t::kTStageCols);
-        for (int i = 0; i < s.nblk; ++i) {
-            const uint4 qv = *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i));
-            uint32_t a[16];
-            q4tm::dequant_block(qv, a);
-            tc_st16(tcol + (uint32_t)(i * q4t::kSlotCols), a);
+        for (int i0 = 0; i0 < s.nblk; i0 += q4t::kQ, ++j) {
+            const int sa = (int)(j % q4t::kRingA);
+            const uint32_t ua = j / q4t::kRingA;
+            if (!waitw(C, P, q4t::kBarAEmpty + sa, (ua & 1u) ^ 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int nq = s.nblk - i0 < q4t::kQ ? s.nblk - i0 : q4t::kQ;
+            for (int ii = 0; ii < nq; ++ii) {
+                const uint4 qv =
+                    *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i0 + ii));
+                uint32_t a[16];
+                q4tm::dequant_block(qv, a);
+                tc_st16(tlane + q4t::a_col(sa, ii), a);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(C.bar(q4t::kBarAFull + sa));
         }
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(C.bar(q4t::kBarAFull + ts));
-            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
-        }
+        if (!ok) break;
+        if (lane == 0) mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
         ++q;
     }
 }
 
-// ---- MMA thread ----
-// Per stage: for each chunk (and hi / lo part) the MMAs of all blocks in turn,
-// so that consecutive MMAs accumulate into different blocks' accumulators.
+// ---- MMA issuers ----
+// Issuer e takes the quads j with j % 2 == e. Per quad: for each 16-value chunk
+// the MMAs of the quad's blocks in turn (consecutive MMAs accumulate into
+// different blocks), then one commit frees the quad's A columns and another
+// hands its accumulators to the epilogue. Every issuer arrives once per stage
+// on the stage's empty barrier: by commit when it read the stage's operands,
+// else directly. One thread issues an MMA about every 50 cycles; two issuers
+// keep the tensor core ahead of the weight stream.
 template <int BT>
-__device__ void run_mma(const Ctx& C, const q4t::Params& P) {
-    constexpr bool kSplit = BT <= 8;
+__device__ void run_mma(const Ctx& C, const q4t::Params& P, int e) {
+    constexpr int kN = q4t::mma_n(BT);
+    constexpr int kRD = q4t::ring_d(BT);
+    constexpr uint32_t kIdesc = q4t::instr_desc(kN);
+    constexpr uint32_t kOpStep = (uint32_t)kN * 32u >> 4;  // descriptor step between operands
     pdl_wait();  // the activations come after the previous kernel
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0;
-    while (!C.aborted() && wk.next(P, &s)) {
+    uint32_t q = 0, j = 0;
+    bool ok = true;
+    while (ok && !C.aborted() && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        const int ts = (int)(q & 1u);
-        const uint32_t u = q >> 1;
-        if (!wait1(C, P, q4t::kBarXOpFull + st, v & 1u)) break;
-        if (!wait1(C, P, q4t::kBarAFull + ts, u & 1u)) break;
-        tc_fence_after();
-        const uint32_t xs = C.sbase + q4t::stage_xop(st);
-        const uint32_t t0 = C.tmem + (uint32_t)(ts * q4t::kTStageCols);
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-            for (int hl = 0; hl < (kSplit ? 1 : 2); ++hl)
-                for (int i = 0; i < s.nblk; ++i) {
-                    const uint32_t a = t0 + (uint32_t)(i * q4t::kSlotCols);
-                    tc_mma(a + 16, a + 8 * c2,
-                           q4t::smem_desc(xs + q4t::x_operand_off(kSplit, i, c2, hl)),
-                           (c2 | hl) != 0);
+        bool used = false;
+        const uint64_t desc0 = q4t::smem_desc(C.sbase + q4t::stage_xop(st), kN);
+        for (int i0 = 0; i0 < s.nblk; i0 += q4t::kQ, ++j) {
+            if ((int)(j & 1u) != e) continue;
+            if (!used) {
+                if (!wait1(C, P, q4t::kBarXOpFull + st, v & 1u)) {
+                    ok = false;
+                    break;
                 }
-        tc_commit(C.bar(q4t::kBarDFull + ts));
-        tc_commit(C.bar(q4t::kBarStageEmpty + st));
+                used = true;
+            }
+            const int sa = (int)(j % q4t::kRingA), sd = (int)(j % kRD);
+            const uint32_t ua = j / q4t::kRingA, ud = j / kRD;
+            if (!wait1(C, P, q4t::kBarAFull + sa, ua & 1u) ||
+                !wait1(C, P, q4t::kBarDEmpty + sd, (ud & 1u) ^ 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int nq = s.nblk - i0 < q4t::kQ ? s.nblk - i0 : q4t::kQ;
+            const uint32_t a0 = C.tmem + q4t::a_col(sa, 0);
+            const uint32_t d0 = C.tmem + q4t::d_col(BT, sd, 0);
+            // operand of block i0 + ii, chunk c2: desc0 + (2 (i0 + ii) + c2) * kOpStep
+            const uint64_t dq = desc0 + (uint64_t)(2 * i0) * kOpStep;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                for (int ii = 0; ii < q4t::kQ; ++ii)
+                    if (ii < nq)
+                        tc_mma(d0 + (uint32_t)(ii * kN), a0 + (uint32_t)(ii * q4t::kACols + 8 * c2),
+                               dq + (uint64_t)(2 * ii + c2) * kOpStep, kIdesc, c2);
+            tc_commit(C.bar(q4t::kBarAEmpty + sa));
+            tc_commit(C.bar(q4t::kBarDFull + sd));
+        }
+        if (!ok) break;
+        if (used)
+            tc_commit(C.bar(q4t::kBarStageEmpty + st));
+        else
+            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
         ++q;
     }
     // every MMA issued completes before tensor memory is freed
@@ -404,41 +449,43 @@ __device__ __forceinline__ void finish_piece(const q4t::Params& P, const q4t::St
     if (lane == 0) *ticket = 0u;
 }
 
+// acc[t] += d * (hi + lo) of one block's accumulator columns: hi parts of
+// token t in column t, lo parts in column N / 2 + t.
 template <int BT>
-__device__ __forceinline__ void accumulate(float (&acc)[BT], float dd, const uint32_t (&D)[16]) {
-    constexpr bool kSplit = BT <= 8;
+__device__ __forceinline__ void accumulate(float (&acc)[BT], float dd, const uint32_t (&Dh)[16],
+                                           const uint32_t (&Dl)[16]) {
+    constexpr int kHalf = q4t::mma_n(BT) / 2;
 #pragma unroll
     for (int t = 0; t < BT; ++t) {
-        const float val = kSplit ? __uint_as_float(D[t]) + __uint_as_float(D[8 + t])
-                                 : __uint_as_float(D[t]);
-        acc[t] = fmaf(dd, val, acc[t]);
+        const float hi = __uint_as_float(Dh[t]);
+        const float lo = kHalf == 8 ? __uint_as_float(Dh[8 + t]) : __uint_as_float(Dl[t]);
+        acc[t] = fmaf(dd, hi + lo, acc[t]);
     }
 }
 
 template <int BT>
 __device__ void run_epilogue(const Ctx& C, const q4t::Params& P, int ew, int lane) {
+    constexpr int kN = q4t::mma_n(BT);
+    constexpr int kRD = q4t::ring_d(BT);
     const int r = ew * 32 + lane;
     const uint32_t tlane = C.tmem + ((uint32_t)(ew * 32) << 16);
     pdl_wait();  // partial sums, tickets and y are written below
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
     q4t::Stage s;
-    uint32_t q = 0;
+    uint32_t q = 0, j = 0;
+    bool ok = true;
     float acc[BT];
 #pragma unroll
     for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
-    while (!warp_aborted(C) && wk.next(P, &s)) {
+    while (ok && !warp_aborted(C) && wk.next(P, &s)) {
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
-        const int ts = (int)(q & 1u);
-        const uint32_t u = q >> 1;
         if (s.first) {
 #pragma unroll
             for (int t = 0; t < BT; ++t) acc[t] = 0.0f;
         }
         if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;  // the stage's scales
-        if (!waitw(C, P, q4t::kBarDFull + ts, u & 1u)) break;
-        tc_fence_after();
         const q4t::Desc& G = P.g[s.g];
         const int c0 = s.kb0 - q4t::window_of(s.kb0);
         const bool live = (int64_t)s.tile * q4t::kM + r < G.n;
@@ -447,29 +494,39 @@ __device__ void run_epilogue(const Ctx& C, const q4t::Params& P, int ew, int lan
             G.d_box ? reinterpret_cast<const uint16_t*>(dsm + r * 16) + c0
                     : reinterpret_cast<const uint16_t*>(
                           dsm + r * q4t::kDSlot + q4t::d_copy(G, s.tile, s.kb0, s.nblk, r).lead);
-        const uint32_t tcol = tlane + (uint32_t)(ts * q4t::kTStageCols) + 16u;
-        for (int i0 = 0; i0 < s.nblk; i0 += 4) {
-            uint32_t D0[16], D1[16], D2[16], D3[16];
-            tc_ld16(tcol + (uint32_t)(i0 * q4t::kSlotCols), D0);
-            if (i0 + 1 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 1) * q4t::kSlotCols), D1);
-            if (i0 + 2 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 2) * q4t::kSlotCols), D2);
-            if (i0 + 3 < s.nblk) tc_ld16(tcol + (uint32_t)((i0 + 3) * q4t::kSlotCols), D3);
-            tc_wait_ld();
-            const float d0 = live ? __half2float(__ushort_as_half(drow[i0])) : 0.0f;
-            accumulate<BT>(acc, d0, D0);
-            if (i0 + 1 < s.nblk)
-                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 1])) : 0.0f, D1);
-            if (i0 + 2 < s.nblk)
-                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 2])) : 0.0f, D2);
-            if (i0 + 3 < s.nblk)
-                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i0 + 3])) : 0.0f, D3);
+        for (int i0 = 0; i0 < s.nblk; i0 += q4t::kQ, ++j) {
+            const int sd = (int)(j % kRD);
+            const uint32_t ud = j / kRD;
+            if (!waitw(C, P, q4t::kBarDFull + sd, ud & 1u)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int nq = s.nblk - i0 < q4t::kQ ? s.nblk - i0 : q4t::kQ;
+            // two blocks per round: their columns, one wait, then the math
+            for (int ii = 0; ii < nq; ii += 2) {
+                uint32_t H0[16], L0[16], H1[16], L1[16];
+                const uint32_t c = tlane + q4t::d_col(BT, sd, ii);
+                tc_ld16(c, H0);
+                if (kN == 32) tc_ld16(c + 16u, L0);
+                if (ii + 1 < nq) {
+                    tc_ld16(c + (uint32_t)kN, H1);
+                    if (kN == 32) tc_ld16(c + (uint32_t)kN + 16u, L1);
+                }
+                tc_wait_ld();
+                const int i = i0 + ii;
+                accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i])) : 0.0f, H0, L0);
+                if (ii + 1 < nq)
+                    accumulate<BT>(acc, live ? __half2float(__ushort_as_half(drow[i + 1])) : 0.0f, H1,
+                                   L1);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(C.bar(q4t::kBarDEmpty + sd));
         }
-        tc_fence_before();
+        if (!ok) break;
         __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(C.bar(q4t::kBarTEmpty + ts));
-            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
-        }
+        if (lane == 0) mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
         ++q;
         if (s.last) finish_piece<BT>(P, s, ew, lane, acc);
     }
@@ -494,12 +551,15 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
             mbar_init(b + q4t::kBarXOpFull + st, q4t::kArrivalsXOpFull);
             mbar_init(b + q4t::kBarStageEmpty + st, q4t::kArrivalsStageEmpty);
         }
-        for (int ts = 0; ts < q4t::kTStages; ++ts) {
-            mbar_init(b + q4t::kBarAFull + ts, q4t::kArrivalsAFull);
-            mbar_init(b + q4t::kBarDFull + ts, 1);
-            mbar_init(b + q4t::kBarTEmpty + ts, q4t::kArrivalsTEmpty);
+        for (int k = 0; k < q4t::kRingA; ++k) {
+            mbar_init(b + q4t::kBarAFull + k, q4t::kArrivalsAFull);
+            mbar_init(b + q4t::kBarAEmpty + k, 1);
         }
-        mbar_init(b + q4t::kBarDone, 1);
+        for (int k = 0; k < q4t::kMaxRingD; ++k) {
+            mbar_init(b + q4t::kBarDFull + k, 1);
+            mbar_init(b + q4t::kBarDEmpty + k, q4t::kArrivalsDEmpty);
+        }
+        mbar_init(b + q4t::kBarDone, q4t::kMmaIssuers);
         // the swizzled code box needs a 1024-byte aligned destination
         *C.abort_flag = (C.sbase & 1023u) ? 1 : 0;
         if (C.sbase & 1023u) atomicOr(P.ws, kTimeoutFlag);
@@ -530,7 +590,7 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
     } else if (warp == q4t::kProdWarp) {
         run_producer<BT>(C, P, lane);
     } else {
-        if (lane == 0) run_mma<BT>(C, P);
+        if (lane == 0) run_mma<BT>(C, P, warp - q4t::kMmaWarp0);
         __syncwarp();
     }
 

@@ -29,10 +29,15 @@
 //           bytes, else one 16-byte aligned bulk copy per row into a 32-byte
 //           slot per row (the stage's scales at an offset inside it)
 //
-// Tensor memory (512 columns x 128 lanes) holds two tensor stages of kS blocks;
-// block i of tensor stage ts uses columns ts * 256 + 32 i: [0, 16) the A operand
-// (row r = lane r, the block's 32 values (q - 8) as bf16 pairs), [16, 32) its
-// accumulator D (128 x 16, binary32).
+// Tensor memory (512 columns x 128 lanes) holds two rings, both in quads of
+// kQ = 4 blocks (a stage is one or two quads): the A ring, kRingA quads of
+// 4 x 16 columns (row r = lane r, a block's 32 values (q - 8) as bf16 pairs),
+// freed as soon as the quad's MMAs complete; and the D ring, ring_d quads of
+// 4 x N columns (each block's accumulator, 128 x N binary32), freed when the
+// epilogue has read it. N = 16 up to 8 tokens (hi parts of token t in column
+// t, lo parts in 8 + t), N = 32 above (hi in t, lo in 16 + t): one MMA per
+// 16-value chunk and block either way, since an MMA's cost does not grow with
+// N up to 256.
 #pragma once
 
 #include <cuda.h>
@@ -49,17 +54,16 @@
 namespace q4t {
 
 constexpr int kM = 128;        // rows per tile (MMA M)
-constexpr int kN = 16;         // MMA N
 constexpr int kS = 8;          // K blocks per window (and at most per stage)
+constexpr int kQ = 4;          // blocks per tensor-memory quad
 constexpr int kStages = 4;     // shared-memory ring depth
-constexpr int kTStages = 2;    // tensor-memory stages
-constexpr int kSlotCols = 32;  // tensor-memory columns per block
-constexpr int kTStageCols = kS * kSlotCols;     // 256
-constexpr int kTmemCols = kTStages * kTStageCols;  // 512
+constexpr int kACols = 16;     // tensor-memory columns of one block's A operand
+constexpr int kRingA = 4;      // A quads
+constexpr int kTmemCols = 512;
 constexpr int kMaxTokens = 16;
 constexpr int kCodesBytes = kM * 128;               // 16 KB
 constexpr int kXRawBytes = kMaxTokens * kS * 32 * 4;  // 16 KB
-constexpr int kBlockXBytes = 2048;                  // 2 chunks x (hi, lo) x 512 B
+constexpr int kBlockXBytes = 2048;                  // 2 chunks x 32 rows x 32 B
 constexpr int kXOpBytes = kS * kBlockXBytes;        // 16 KB
 constexpr int kDSlot = 32;                          // bytes per row (per-row copies)
 constexpr int kDBytes = kM * kDSlot;                // 4 KB
@@ -72,30 +76,45 @@ constexpr int kDequantWarp0 = 0;  // 4 warps: codes -> (q - 8) bf16 into tensor 
 constexpr int kEpiWarp0 = 4;      // 4 warps: accumulators x scale, partial sums, y
 constexpr int kXWarp0 = 8;        // 4 warps: xraw -> bf16 hi/lo B operands
 constexpr int kProdWarp = 12;     // TMA loads (lane 0) and per-row scale copies (all lanes)
-constexpr int kMmaWarp = 13;      // 1 thread: tcgen05.mma issue
-constexpr int kWarps = 14;
+constexpr int kMmaWarp0 = 13;     // 2 warps, one thread each: tcgen05.mma issue, quads
+                                  // alternating between them
+constexpr int kMmaIssuers = 2;
+constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled box");
+static_assert(kS == 2 * kQ, "a stage is one or two quads");
+
+// MMA N, D quads, and tensor-memory columns for a launch compiled for BT tokens.
+Q4T_HD constexpr int mma_n(int bt) { return bt <= 8 ? 16 : 32; }
+Q4T_HD constexpr int ring_d(int bt) { return (kTmemCols - kRingA * kQ * kACols) / (kQ * mma_n(bt)); }
+Q4T_HD constexpr uint32_t a_col(int slot, int i) { return (uint32_t)((slot * kQ + i) * kACols); }
+Q4T_HD constexpr uint32_t d_col(int bt, int slot, int i) {
+    return (uint32_t)(kRingA * kQ * kACols + (slot * kQ + i) * mma_n(bt));
+}
+static_assert(ring_d(2) == 4 && ring_d(16) == 2, "tensor-memory rings");
 
 // barrier indices (uint64 words at the start of shared memory)
+constexpr int kMaxRingD = 4;
 constexpr int kBarFull = 0;                          // [kStages] every TMA byte of the stage
 constexpr int kBarXOpFull = kBarFull + kStages;      // [kStages] B operands written
 constexpr int kBarStageEmpty = kBarXOpFull + kStages;  // [kStages]
-constexpr int kBarAFull = kBarStageEmpty + kStages;  // [kTStages]
-constexpr int kBarDFull = kBarAFull + kTStages;      // [kTStages]
-constexpr int kBarTEmpty = kBarDFull + kTStages;     // [kTStages]
-constexpr int kBarDone = kBarTEmpty + kTStages;      // 1
+constexpr int kBarAFull = kBarStageEmpty + kStages;  // [kRingA] A quad written
+constexpr int kBarAEmpty = kBarAFull + kRingA;       // [kRingA] A quad's MMAs done
+constexpr int kBarDFull = kBarAEmpty + kRingA;       // [kMaxRingD] D quad's MMAs done
+constexpr int kBarDEmpty = kBarDFull + kMaxRingD;    // [kMaxRingD] D quad read
+constexpr int kBarDone = kBarDEmpty + kMaxRingD;     // 1
 constexpr int kNumBars = kBarDone + 1;
 constexpr int kTmemAddrOff = 8 * kNumBars;  // uint32 written by tcgen05.alloc
 constexpr int kAbortOff = kTmemAddrOff + 4;  // int32 abort flag
 static_assert(kAbortOff + 4 <= kHeaderBytes, "header");
 
 // arrivals per barrier phase
-constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 4 + 1;  // dequant, x, epilogue warps; MMA commit
+constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 4 + kMmaIssuers;  // dequant, x, epilogue
+                                                                   // warps; MMA issuers
 constexpr uint32_t kArrivalsXOpFull = 4;
 constexpr uint32_t kArrivalsAFull = 4;
-constexpr uint32_t kArrivalsTEmpty = 4;
+constexpr uint32_t kArrivalsDEmpty = 4;
 
 Q4T_HD uint32_t stage_base(int st) { return (uint32_t)(kHeaderBytes + st * kStageBytes); }
 Q4T_HD uint32_t stage_codes(int st) { return stage_base(st); }
@@ -106,22 +125,18 @@ Q4T_HD uint32_t stage_d(int st) { return stage_base(st) + kCodesBytes + kXRawByt
 // Code bytes of block c (0..kS-1) of the window, row r, inside the swizzled box.
 Q4T_HD uint32_t code_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// Byte offset, inside a stage's operand region, of the 16-byte row holding MMA
-// positions [8 hh, 8 hh + 8) of chunk c2 (16 K values) of stage block i for
-// MMA row `row` (0..15) of operand part `hl` (0 = hi, 1 = lo). With at most 8
-// tokens (split) the hi parts of tokens t are rows t and the lo parts rows
-// 8 + t of one 16-row operand (1 KB per block); with more tokens the hi and lo
-// parts are two 16-row operands (2 KB per block) accumulated into the same D.
-// Inside one 16 x 16 operand: core matrix (row group g = row / 8, K half hh) at
-// hh * 256 + g * 128, row r % 8 at 16 (r % 8).
-constexpr uint32_t kLBO = 256;  // between the two K halves of an operand
-constexpr uint32_t kSBO = 128;  // between the two 8-row groups
-Q4T_HD uint32_t x_operand_off(bool split, int i, int c2, int hl) {
-    return split ? (uint32_t)(i * 1024 + c2 * 512) : (uint32_t)(i * 2048 + c2 * 1024 + hl * 512);
-}
-Q4T_HD uint32_t x_row_off(bool split, int i, int c2, int hh, int t, int hl) {
-    const int row = split ? (hl ? 8 + t : t) : t;
-    return x_operand_off(split, i, c2, hl) + (uint32_t)(hh * kLBO) + (uint32_t)((row >> 3) * kSBO) +
+// Byte offset, inside a stage's operand region, of the N x 16 bf16 B operand
+// of chunk c2 (16 K values) of stage block i, and of the 16-byte row holding
+// its MMA positions [8 hh, 8 hh + 8) for token t, part hl (0 = hi, 1 = lo):
+// operand row t (hi) or N / 2 + t (lo). Inside an operand: core matrix (row
+// group g = row / 8, K half hh) at hh * LBO + g * 128 with LBO = N * 16, row
+// r % 8 at 16 (r % 8).
+constexpr uint32_t kSBO = 128;  // between 8-row groups
+Q4T_HD uint32_t lbo(int n) { return (uint32_t)(n * 16); }
+Q4T_HD uint32_t x_operand_off(int n, int i, int c2) { return (uint32_t)((2 * i + c2) * n * 32); }
+Q4T_HD uint32_t x_row_off(int n, int i, int c2, int hh, int t, int hl) {
+    const int row = hl ? n / 2 + t : t;
+    return x_operand_off(n, i, c2) + (uint32_t)hh * lbo(n) + (uint32_t)((row >> 3) * kSBO) +
            (uint32_t)((row & 7) * 16);
 }
 
@@ -137,17 +152,18 @@ Q4T_HD int element_at(int kappa) {
 }
 
 // tcgen05.mma instruction descriptor: kind::f16, A and B bf16, D binary32,
-// both K-major, M = 128, N = 16.
-constexpr uint32_t kInstrDesc = (1u << 4)            // D format F32
-                                | (1u << 7)          // A format BF16
-                                | (1u << 10)         // B format BF16
-                                | ((uint32_t)(kN >> 3) << 17)
-                                | ((uint32_t)(kM >> 4) << 24);
+// both K-major, M = 128, N = n.
+Q4T_HD constexpr uint32_t instr_desc(int n) {
+    return (1u << 4)      // D format F32
+           | (1u << 7)    // A format BF16
+           | (1u << 10)   // B format BF16
+           | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+}
 
-// Shared-memory matrix descriptor of one 16 x 16 bf16 B operand at byte
-// address `addr` (canonical K-major layout, no swizzle).
-Q4T_HD uint64_t smem_desc(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((kLBO >> 4) & 0x3FFFu) << 16) |
+// Shared-memory matrix descriptor of one n x 16 bf16 B operand at byte address
+// `addr` (canonical K-major layout, no swizzle).
+Q4T_HD uint64_t smem_desc(uint32_t addr, int n) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo(n) >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((kSBO >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
 }
 
