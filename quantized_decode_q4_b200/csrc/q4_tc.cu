@@ -97,14 +97,16 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(idesc), "r"(0u)
         : "memory");
 }
+// No memory clobber: the store writes tensor memory only, and as a volatile asm
+// it stays ordered with the wait, fence and barrier asm that publish it, while
+// shared-memory loads of later blocks may move above it.
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
         "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
         "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-        "r"(v[15])
-        : "memory");
+        "r"(v[15]));
 }
 __device__ __forceinline__ void tc_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -320,12 +322,20 @@ __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane
             }
             tc_fence_after();
             const int nq = s.nblk - i0 < q4t::kQ ? s.nblk - i0 : q4t::kQ;
-            for (int ii = 0; ii < nq; ++ii) {
-                const uint4 qv =
-                    *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i0 + ii));
-                uint32_t a[16];
-                q4tm::dequant_block(qv, a);
-                tc_st16(tlane + q4t::a_col(sa, ii), a);
+            // the quad's code bytes first (one 16-byte load per block), then the
+            // blocks' operands
+            uint4 qv[q4t::kQ];
+#pragma unroll
+            for (int ii = 0; ii < q4t::kQ; ++ii)
+                qv[ii] = ii < nq ? *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i0 + ii))
+                                 : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int ii = 0; ii < q4t::kQ; ++ii) {
+                if (ii < nq) {
+                    uint32_t a[16];
+                    q4tm::dequant_block(qv[ii], a);
+                    tc_st16(tlane + q4t::a_col(sa, ii), a);
+                }
             }
             tc_wait_st();
             tc_fence_before();
