@@ -451,6 +451,8 @@ q4_status stack_groups(const q4_stack* s, std::vector<std::pair<int, int>>* out)
 
 // Validate a stack; returns the ticket region shared by all groups and the
 // workspace bytes needed.
+// Validate a stack; returns the ticket region shared by all groups and the
+// workspace bytes needed.
 q4_status stack_check(const q4_stack* s, int b, std::vector<std::pair<int, int>>* groups,
                       int64_t* tickets, size_t* need) {
     q4_status st = stack_groups(s, groups);

@@ -2,19 +2,20 @@
 //
 // "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
 // section 3 "Dequantizzazione Integrata": the decode mat-vec dequantises in
-// registers. One CTA per SM walks a contiguous range of units (4 rows of one
-// GEMV over one K split). Each warp streams its units' code bytes and binary16
-// scales from HBM through a private ring of shared-memory stages filled by bulk
-// copies on the TMA engine (one mbarrier per stage; a stage is refilled as soon
-// as the warp has read it), so the weight stream never waits for the math. The
-// activations of a (GEMV, split) segment are staged once per CTA. Nibbles are
-// unpacked to exact binary32 (q - 8) in registers and accumulated with packed
-// f32x2 FMAs; the binary16 scale is applied once per 32 weights; rows are
-// reduced with warp shuffles. When K is split, the warp that completes a row
-// tile last adds the partial sums in split order (deterministic).
-// The first chunks are requested before the wait on the previous kernel
-// (programmatic dependent launch), so consecutive launches overlap their weight
-// streams.
+// registers. One CTA per SM walks a contiguous range of the group's row space
+// (rows of (GEMV, K split) segments laid end to end). Each warp streams its
+// tiles' code bytes and binary16 scales from HBM through a private ring of
+// shared-memory stages filled by bulk copies on the TMA engine (one mbarrier per
+// stage; a stage is refilled as soon as the warp has read it), so the weight
+// stream never waits for the math. The activations of a (GEMV, split) segment
+// are staged once per CTA in 24-bit block fixed point; each block's dot product
+// is exact in integers (dp4a over the three digit planes) and its binary16 and
+// activation scales are applied once per 32 weights; rows are reduced with warp
+// shuffles. When K is split, the warp that completes a row tile last adds the
+// partial sums in split order (deterministic).
+// One dependency group per launch: the first tiles are requested before the
+// wait on the previous kernel (programmatic dependent launch), so consecutive
+// launches overlap their weight streams.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -32,25 +33,61 @@ namespace {
 
 constexpr uint32_t kTimeoutFlag = 1u;
 
+// The kernel's source of groups: one dependency group per launch (a whole
+// stack in one launch with a software grid barrier between groups measured
+// slower on B200 than programmatic dependent launch of one kernel per group).
+struct OneGroup {
+    const q4s::Params& P;
+    __device__ int groups() const { return 1; }
+    __device__ q4s::View view(int) const {
+        q4s::View v;
+        v.g = P.g;
+        v.count = P.count;
+        v.total_rows = P.total_rows;
+        return v;
+    }
+    __device__ uint32_t* ws() const { return P.ws; }
+};
+
 // Copy issuer of one warp: walks the warp's tiles in the same order as the math
-// loop and issues each tile's copies (two requests when K is not split: all
+// loop, group after group (the weights do not wait for the barrier between
+// groups), and issues each tile's copies (two requests when K is not split: all
 // codes, all scales) into the next stage.
+template <class Src>
 struct Issuer {
     q4s::Walk wk;
+    q4s::View v;                 // the current group
     int64_t row0;                // first row of the next tile to issue
+    int gi, ngroups, warp;
     bool has;                    // a tile is pending
 
     __device__ bool done() const { return !has; }
 
-    __device__ void begin(const q4s::Params& P, int64_t lo, int64_t hi, int warp) {
-        wk.begin(lo, hi, warp);
-        has = wk.next_piece(P);
-        if (has) row0 = wk.wr;
+    __device__ void start(const Src& S) {
+        for (; gi < ngroups; ++gi) {
+            v = S.view(gi);
+            int64_t lo, hi;
+            q4s::cta_range(v, blockIdx.x, gridDim.x, &lo, &hi);
+            wk.begin(lo, hi, warp);
+            has = wk.next_piece(v);
+            if (has) {
+                row0 = wk.wr;
+                return;
+            }
+        }
+        has = false;
+    }
+
+    __device__ void begin(const Src& S, int w) {
+        warp = w;
+        gi = 0;
+        ngroups = S.groups();
+        start(S);
     }
 
     // issue the pending tile into `stage` (whole warp), then advance
-    __device__ void issue(const q4s::Params& P, uint8_t* stage_base, uint64_t* bar, int lane) {
-        const q4s::Desc& G = P.g[wk.g];
+    __device__ void issue(const Src& S, uint8_t* stage_base, uint64_t* bar, int lane) {
+        const q4s::Desc& G = v.g[wk.g];
         const int64_t left = wk.wend - row0;
         const int rows = left < q4s::kRows ? (int)left : q4s::kRows;
         const q4s::LaneCopy c = q4s::lane_copy(G, wk.split, row0, rows, lane);
@@ -64,23 +101,28 @@ struct Issuer {
                      bar);
         row0 += q4s::kRows;
         if (row0 >= wk.wend) {
-            has = wk.next_piece(P);
-            if (has) row0 = wk.wr;
+            has = wk.next_piece(v);
+            if (has) {
+                row0 = wk.wr;
+            } else {
+                ++gi;
+                start(S);
+            }
         }
     }
 };
 
-__device__ __forceinline__ void wait_stage(const q4s::Params& P, uint64_t* bar, uint32_t parity,
-                                           int lane) {
+__device__ __forceinline__ void wait_stage(uint32_t* ws, uint64_t* bar, uint32_t parity, int lane) {
     if (!mbar_wait_bounded(bar, parity)) {
-        if (lane == 0) atomicOr(P.ws, kTimeoutFlag);
+        if (lane == 0) atomicOr(ws, kTimeoutFlag);
         mbar_wait_bounded(bar, parity);
     }
 }
 
 // Stage the activations of split `split` of GEMV `G` in 24-bit block fixed
 // point (all threads of the CTA). Warp w quantises blocks w, w + kWarps, ...;
-// lane l holds element l of the block. All loads are issued first.
+// lane l holds element l of the block. All loads are issued first; they read
+// L2 (the activations may have been written by another CTA of this launch).
 __device__ __forceinline__ void stage_x(const q4s::Desc& G, int split, uint4* xq, int warp,
                                         int lane) {
     constexpr int kPer = (q4s::kMaxSplitBlocks + q4s::kWarps - 1) / q4s::kWarps;
@@ -90,7 +132,7 @@ __device__ __forceinline__ void stage_x(const q4s::Desc& G, int split, uint4* xq
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int j = warp + i * q4s::kWarps;
-        v[i] = j < kbs ? xg[j * 32 + lane] : 0.0f;
+        v[i] = j < kbs ? __ldcg(xg + j * 32 + lane) : 0.0f;
     }
     uint8_t* xb = reinterpret_cast<uint8_t*>(xq);
 #pragma unroll
@@ -121,7 +163,7 @@ __device__ __forceinline__ void stage_x(const q4s::Desc& G, int split, uint4* xq
 // Finish one tile: reduce each row over the lanes; lane r stores row r, or,
 // with a split K, stores its partial sum and, if it is the last split of the
 // row to arrive, adds the partials in split order and resets the row's ticket.
-__device__ __forceinline__ void finish_tile(const q4s::Params& P, const q4s::Desc& G, int split,
+__device__ __forceinline__ void finish_tile(uint32_t* ws, const q4s::Desc& G, int split,
                                             int64_t row0, int rows,
                                             const float (&acc)[q4s::kRows], int lane) {
     // all rows' butterflies interleaved, then lane r keeps row r
@@ -142,29 +184,26 @@ __device__ __forceinline__ void finish_tile(const q4s::Params& P, const q4s::Des
         G.y[row] = mine;
         return;
     }
-    float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
+    float* part = reinterpret_cast<float*>(ws) + G.part_off;
     part[(int64_t)split * G.n + row] = mine;
     __threadfence();
-    const uint32_t t = atomicAdd(P.ws + G.ticket_off + row, 1u);
+    const uint32_t t = atomicAdd(ws + G.ticket_off + row, 1u);
     if (t != (uint32_t)G.splits - 1u) return;
     __threadfence();
     float s = 0.0f;
     for (int sp = 0; sp < G.splits; ++sp) s += __ldcg(part + (int64_t)sp * G.n + row);
     G.y[row] = s;
-    P.ws[G.ticket_off + row] = 0u;
+    ws[G.ticket_off + row] = 0u;
 }
 
-}  // namespace
-
-__global__ void __launch_bounds__(q4s::kThreads, Q4_STREAM_MINB)
-    gemv_stream_kernel(const __grid_constant__ q4s::Params P) {
+template <class Src>
+__device__ __forceinline__ void stream_body(const Src& S) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw) + warp * q4s::kStages;
     uint4* xq = reinterpret_cast<uint4*>(smem_raw + q4s::kBarBytes);
     uint8_t* ring = smem_raw + q4s::stage_offset(warp, 0);
-    int64_t lo, hi;
-    q4s::cta_range(P, blockIdx.x, gridDim.x, &lo, &hi);
+    uint32_t* ws = S.ws();
 
     if (lane == 0) {
         for (int s = 0; s < q4s::kStages; ++s) mbar_init(bars + s, 1);
@@ -173,94 +212,112 @@ __global__ void __launch_bounds__(q4s::kThreads, Q4_STREAM_MINB)
     __syncwarp();
 
     // the copy issuer runs kStages tiles ahead of the math
-    Issuer is;
-    is.begin(P, lo, hi, warp);
+    Issuer<Src> is;
+    is.begin(S, warp);
     for (int s = 0; s < q4s::kStages && !is.done(); ++s)
-        is.issue(P, ring + s * q4s::kStageBytes, bars + s, lane);
+        is.issue(S, ring + s * q4s::kStageBytes, bars + s, lane);
 
     // warm L2 with the activations of the first piece (a hint only: the reads
     // that use them come after the wait on the previous kernel)
-    if (lo < hi && warp == 0 && lane == 0) {
-        const q4s::Where w0 = q4s::locate(P, lo);
-        const q4s::Desc& G0 = P.g[w0.g];
-        bulk_prefetch_l2(G0.x + (int64_t)w0.split * G0.nb_split * 32,
-                         (uint32_t)q4s::split_blocks(G0, w0.split) * 128u);
+    {
+        const q4s::View v0 = S.view(0);
+        int64_t lo0, hi0;
+        q4s::cta_range(v0, blockIdx.x, gridDim.x, &lo0, &hi0);
+        if (lo0 < hi0 && warp == 0 && lane == 0) {
+            const q4s::Where w0 = q4s::locate(v0, lo0);
+            const q4s::Desc& G0 = v0.g[w0.g];
+            bulk_prefetch_l2(G0.x + (int64_t)w0.split * G0.nb_split * 32,
+                             (uint32_t)q4s::split_blocks(G0, w0.split) * 128u);
+        }
     }
 
     pdl_launch_dependents();
     pdl_wait();
 
     uint32_t stage = 0, parity = 0;
-    int64_t pos = lo;
-    while (pos < hi) {
-        const q4s::Where w = q4s::locate(P, pos);
-        const int64_t p1 = w.seg_end < hi ? w.seg_end : hi;
-        const int64_t seg_row0 = pos - w.row;
-        const q4s::Desc& G = P.g[w.g];
-        __syncthreads();  // every warp is done with the previous activations
-        stage_x(G, w.split, xq, warp, lane);
-        __syncthreads();
-        const int kbs = q4s::split_blocks(G, w.split);
-        const int nsub = (kbs + 31) >> 5;
-        const uint4* xl = xq + lane;
-        int64_t ra, rb;
-        q4s::warp_rows(pos, p1, warp, &ra, &rb);
-        for (int64_t row0 = ra - seg_row0; row0 < rb - seg_row0; row0 += q4s::kRows) {
-            const int64_t left = rb - seg_row0 - row0;
-            const int rows = left < q4s::kRows ? (int)left : q4s::kRows;
-            uint8_t* st = ring + stage * q4s::kStageBytes;
-            const uint8_t* qrow[q4s::kRows];
-            const uint8_t* drow[q4s::kRows];
+    for (int gi = 0; gi < S.groups(); ++gi) {
+        const q4s::View V = S.view(gi);
+        int64_t lo, hi;
+        q4s::cta_range(V, blockIdx.x, gridDim.x, &lo, &hi);
+        int64_t pos = lo;
+        while (pos < hi) {
+            const q4s::Where w = q4s::locate(V, pos);
+            const int64_t p1 = w.seg_end < hi ? w.seg_end : hi;
+            const int64_t seg_row0 = pos - w.row;
+            const q4s::Desc& G = V.g[w.g];
+            __syncthreads();  // every warp is done with the previous activations
+            stage_x(G, w.split, xq, warp, lane);
+            __syncthreads();
+            const int kbs = q4s::split_blocks(G, w.split);
+            const int nsub = (kbs + 31) >> 5;
+            const uint4* xl = xq + lane;
+            int64_t ra, rb;
+            q4s::warp_rows(pos, p1, warp, &ra, &rb);
+            for (int64_t row0 = ra - seg_row0; row0 < rb - seg_row0; row0 += q4s::kRows) {
+                const int64_t left = rb - seg_row0 - row0;
+                const int rows = left < q4s::kRows ? (int)left : q4s::kRows;
+                uint8_t* st = ring + stage * q4s::kStageBytes;
+                const uint8_t* qrow[q4s::kRows];
+                const uint8_t* drow[q4s::kRows];
 #pragma unroll
-            for (int r = 0; r < q4s::kRows; ++r) {
-                uint32_t qo, dof;
-                q4s::row_read_offsets(G, w.split, row0, rows, r, &qo, &dof);
-                qrow[r] = st + qo + lane * 16;
-                drow[r] = st + dof + lane * 2;
-            }
-            float acc[q4s::kRows];
+                for (int r = 0; r < q4s::kRows; ++r) {
+                    uint32_t qo, dof;
+                    q4s::row_read_offsets(G, w.split, row0, rows, r, &qo, &dof);
+                    qrow[r] = st + qo + lane * 16;
+                    drow[r] = st + dof + lane * 2;
+                }
+                float acc[q4s::kRows];
 #pragma unroll
-            for (int r = 0; r < q4s::kRows; ++r) acc[r] = 0.0f;
-            wait_stage(P, bars + stage, parity, lane);
-            for (int sub = 0; sub < nsub; ++sub) {
-                if ((sub << 5) + lane < kbs) {
-                    const uint4* xe = xl + ((sub * q4s::kXEntries) << 5);
-                    q4dev::XDigits xd;
-                    const uint4 a0 = xe[0 << 5], a1 = xe[1 << 5], b0 = xe[2 << 5],
-                                b1 = xe[3 << 5], c0 = xe[4 << 5], c1 = xe[5 << 5], k = xe[6 << 5];
-                    xd.a[0] = a0.x; xd.a[1] = a0.y; xd.a[2] = a0.z; xd.a[3] = a0.w;
-                    xd.a[4] = a1.x; xd.a[5] = a1.y; xd.a[6] = a1.z; xd.a[7] = a1.w;
-                    xd.b[0] = b0.x; xd.b[1] = b0.y; xd.b[2] = b0.z; xd.b[3] = b0.w;
-                    xd.b[4] = b1.x; xd.b[5] = b1.y; xd.b[6] = b1.z; xd.b[7] = b1.w;
-                    xd.c[0] = c0.x; xd.c[1] = c0.y; xd.c[2] = c0.z; xd.c[3] = c0.w;
-                    xd.c[4] = c1.x; xd.c[5] = c1.y; xd.c[6] = c1.z; xd.c[7] = c1.w;
-                    const float sx = __uint_as_float(k.w);
+                for (int r = 0; r < q4s::kRows; ++r) acc[r] = 0.0f;
+                wait_stage(ws, bars + stage, parity, lane);
+                for (int sub = 0; sub < nsub; ++sub) {
+                    if ((sub << 5) + lane < kbs) {
+                        const uint4* xe = xl + ((sub * q4s::kXEntries) << 5);
+                        q4dev::XDigits xd;
+                        const uint4 a0 = xe[0 << 5], a1 = xe[1 << 5], b0 = xe[2 << 5],
+                                    b1 = xe[3 << 5], c0 = xe[4 << 5], c1 = xe[5 << 5],
+                                    k = xe[6 << 5];
+                        xd.a[0] = a0.x; xd.a[1] = a0.y; xd.a[2] = a0.z; xd.a[3] = a0.w;
+                        xd.a[4] = a1.x; xd.a[5] = a1.y; xd.a[6] = a1.z; xd.a[7] = a1.w;
+                        xd.b[0] = b0.x; xd.b[1] = b0.y; xd.b[2] = b0.z; xd.b[3] = b0.w;
+                        xd.b[4] = b1.x; xd.b[5] = b1.y; xd.b[6] = b1.z; xd.b[7] = b1.w;
+                        xd.c[0] = c0.x; xd.c[1] = c0.y; xd.c[2] = c0.z; xd.c[3] = c0.w;
+                        xd.c[4] = c1.x; xd.c[5] = c1.y; xd.c[6] = c1.z; xd.c[7] = c1.w;
+                        const float sx = __uint_as_float(k.w);
 #pragma unroll
-                    for (int r = 0; r < q4s::kRows; ++r) {
-                        const uint4 q = *reinterpret_cast<const uint4*>(qrow[r] + sub * 512);
-                        const float dd =
-                            __half2float(*reinterpret_cast<const __half*>(drow[r] + sub * 64));
-                        const float v = q4dev::block_dot_int(q, xd, (int32_t)k.x, (int32_t)k.y,
-                                                             (int32_t)k.z);
-                        acc[r] = fmaf(dd * sx, v, acc[r]);
+                        for (int r = 0; r < q4s::kRows; ++r) {
+                            const uint4 q = *reinterpret_cast<const uint4*>(qrow[r] + sub * 512);
+                            const float dd = __half2float(
+                                *reinterpret_cast<const __half*>(drow[r] + sub * 64));
+                            const float v = q4dev::block_dot_int(q, xd, (int32_t)k.x,
+                                                                 (int32_t)k.y, (int32_t)k.z);
+                            acc[r] = fmaf(dd * sx, v, acc[r]);
+                        }
                     }
                 }
+                __syncwarp();
+                if (!is.done()) {
+                    // the stage is free: refill it kStages tiles ahead (the proxy fence
+                    // orders this warp's reads before the async writes)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    is.issue(S, st, bars + stage, lane);
+                }
+                if (++stage == q4s::kStages) {
+                    stage = 0;
+                    parity ^= 1u;
+                }
+                finish_tile(ws, G, w.split, row0, rows, acc, lane);
             }
-            __syncwarp();
-            if (!is.done()) {
-                // the stage is free: refill it kStages tiles ahead (the proxy fence
-                // orders this warp's reads before the async writes)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                is.issue(P, st, bars + stage, lane);
-            }
-            if (++stage == q4s::kStages) {
-                stage = 0;
-                parity ^= 1u;
-            }
-            finish_tile(P, G, w.split, row0, rows, acc, lane);
+            pos = p1;
         }
-        pos = p1;
     }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(q4s::kThreads, Q4_STREAM_MINB)
+    gemv_stream_kernel(const __grid_constant__ q4s::Params P) {
+    stream_body(OneGroup{P});
 }
 
 cudaError_t setup_stream_kernel(int optin_smem) {

@@ -80,6 +80,13 @@ struct Params {
     uint32_t* ws;
 };
 
+// One dependency group as the walks see it (Params has the same members).
+struct View {
+    const Desc* g;
+    int32_t count;
+    int64_t total_rows;
+};
+
 // Segment of a row-space index: GEMV g, split, row within the GEMV, and the end
 // (exclusive, in row space) of the segment.
 struct Where {
@@ -89,7 +96,8 @@ struct Where {
 
 // The row space stays below 2^31 rows (checked by the planner), so this uses
 // 32-bit division.
-Q4S_HD Where locate(const Params& P, int64_t r) {
+template <class PV>
+Q4S_HD Where locate(const PV& P, int64_t r) {
     int g = 0;
     while (g + 1 < P.count && r >= P.g[g + 1].row_begin) ++g;
     const Desc& G = P.g[g];
@@ -108,7 +116,8 @@ Q4S_HD int split_blocks(const Desc& G, int split) {
     return rest < G.nb_split ? rest : G.nb_split;
 }
 
-Q4S_HD void cta_range(const Params& P, int cta, int grid, int64_t* lo, int64_t* hi) {
+template <class PV>
+Q4S_HD void cta_range(const PV& P, int cta, int grid, int64_t* lo, int64_t* hi) {
     const uint64_t R = (uint64_t)P.total_rows;  // < 2^31
     *lo = (int64_t)(R * (uint32_t)cta / (uint32_t)grid);
     *hi = (int64_t)(R * (uint32_t)(cta + 1) / (uint32_t)grid);
@@ -218,7 +227,8 @@ struct Walk {
     }
 
     // advance to the next piece that gives this warp at least one row
-    Q4S_HD bool next_piece(const Params& P) {
+    template <class PV>
+    Q4S_HD bool next_piece(const PV& P) {
         while (pos < hi) {
             const Where w = locate(P, pos);
             const int64_t p1 = w.seg_end < hi ? w.seg_end : hi;
