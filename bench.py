@@ -202,6 +202,26 @@ def reference_arm(args, workload):
 # the CUDA library
 # ---------------------------------------------------------------------------
 
+def profile_gemv(args):
+    """Launches of a single GEMV (synthetic weights packed on the GPU) for profilers."""
+    import torch
+
+    from quantized_decode_q4_b200 import q4, synth
+    n, k = (int(v) for v in args.profile_gemv.split(","))
+    w = synth.matrix(7, 7, n, k, synth.WEIGHT_STD, device="cuda")
+    m = q4.pack(w)
+    del w
+    X = synth.normal(7, 8, 0, args.batch * k, 1.0, device="cuda").view(args.batch, k)
+    Y = torch.empty(args.batch, n, device="cuda")
+    ws = q4.workspace(q4.workspace_bytes(n, k, args.batch))
+    for _ in range(args.warmup + args.steps):
+        q4.gemv_batched(m, X, Y, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_gemv": [n, k], "batch": args.batch,
+                      "launches": args.warmup + args.steps,
+                      "status": q4.workspace_status(ws)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -212,7 +232,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--launch", default="graph", choices=["graph", "direct"])
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--profile-gemv", metavar="N,K", default=None,
+                    help="no bench line: run --warmup + --steps launches of one GEMV of this "
+                         "shape for --batch tokens (a small case for ncu captures)")
     args = ap.parse_args()
+    if args.profile_gemv:
+        profile_gemv(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         ap.error("at least 3 warm-up steps")
 
