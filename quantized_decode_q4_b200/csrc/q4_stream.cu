@@ -11,8 +11,9 @@
 // are staged once per CTA in 24-bit block fixed point; each block's dot product
 // is exact in integers (dp4a over the three digit planes) and its binary16 and
 // activation scales are applied once per 32 weights; rows are reduced with warp
-// shuffles. When K is split, the warp that completes a row tile last adds the
-// partial sums in split order (deterministic).
+// shuffles. Finished rows wait in the lanes and are published 32 at a time; when
+// K is split, the last split of a row to arrive adds the partial sums in split
+// order (deterministic).
 // One dependency group per launch: the first tiles are requested before the
 // wait on the previous kernel (programmatic dependent launch), so consecutive
 // launches overlap their weight streams.
@@ -160,40 +161,41 @@ __device__ __forceinline__ void stage_x(const q4s::Desc& G, int split, uint4* xq
     }
 }
 
-// Finish one tile: reduce each row over the lanes; lane r stores row r, or,
-// with a split K, stores its partial sum and, if it is the last split of the
-// row to arrive, adds the partials in split order and resets the row's ticket.
-__device__ __forceinline__ void finish_tile(uint32_t* ws, const q4s::Desc& G, int split,
-                                            int64_t row0, int rows,
-                                            const float (&acc)[q4s::kRows], int lane) {
-    // all rows' butterflies interleaved, then lane r keeps row r
-    float v[q4s::kRows];
-#pragma unroll
-    for (int r = 0; r < q4s::kRows; ++r) v[r] = acc[r];
+// Sum each of a tile's rows over the lanes (butterflies interleaved); every
+// lane gets every row's total.
+__device__ __forceinline__ void reduce_tile(float (&v)[q4s::kRows]) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
         for (int r = 0; r < q4s::kRows; ++r) v[r] += __shfl_xor_sync(0xffffffffu, v[r], off);
-    float mine = v[0];
-#pragma unroll
-    for (int r = 1; r < q4s::kRows; ++r)
-        if (lane == r) mine = v[r];
-    if (lane >= rows) return;
-    const int64_t row = row0 + lane;
+}
+
+// Publish up to 32 consecutive rows of one (GEMV, split) piece, row
+// brow0 + l held by lane l: store y, or, with a split K, store the partial
+// sums, fence once, take each row's ticket, and let the last split of a row to
+// arrive add the partials in split order and reset the ticket.
+__device__ __forceinline__ void flush_rows(uint32_t* ws, const q4s::Desc& G, int split, int64_t brow0,
+                                           int nbuf, float mine, int lane) {
+    const bool act = lane < nbuf;
+    const int64_t row = brow0 + lane;
     if (G.splits == 1) {
-        G.y[row] = mine;
+        if (act) G.y[row] = mine;
         return;
     }
     float* part = reinterpret_cast<float*>(ws) + G.part_off;
-    part[(int64_t)split * G.n + row] = mine;
+    if (act) part[(int64_t)split * G.n + row] = mine;
     __threadfence();
-    const uint32_t t = atomicAdd(ws + G.ticket_off + row, 1u);
-    if (t != (uint32_t)G.splits - 1u) return;
-    __threadfence();
-    float s = 0.0f;
-    for (int sp = 0; sp < G.splits; ++sp) s += __ldcg(part + (int64_t)sp * G.n + row);
-    G.y[row] = s;
-    ws[G.ticket_off + row] = 0u;
+    bool last = false;
+    if (act) last = atomicAdd(ws + G.ticket_off + row, 1u) == (uint32_t)G.splits - 1u;
+    if (__any_sync(0xffffffffu, last)) {
+        __threadfence();
+        if (last) {
+            float sum = 0.0f;
+            for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
+            G.y[row] = sum;
+            ws[G.ticket_off + row] = 0u;
+        }
+    }
 }
 
 template <class Src>
@@ -253,6 +255,11 @@ __device__ __forceinline__ void stream_body(const Src& S) {
             const uint4* xl = xq + lane;
             int64_t ra, rb;
             q4s::warp_rows(pos, p1, warp, &ra, &rb);
+            // finished rows wait in the lanes (row brow0 + l in lane l) and are
+            // published 32 at a time
+            int64_t brow0 = ra - seg_row0;
+            int nbuf = 0;
+            float mine = 0.0f;
             for (int64_t row0 = ra - seg_row0; row0 < rb - seg_row0; row0 += q4s::kRows) {
                 const int64_t left = rb - seg_row0 - row0;
                 const int rows = left < q4s::kRows ? (int)left : q4s::kRows;
@@ -306,8 +313,18 @@ __device__ __forceinline__ void stream_body(const Src& S) {
                     stage = 0;
                     parity ^= 1u;
                 }
-                finish_tile(ws, G, w.split, row0, rows, acc, lane);
+                reduce_tile(acc);
+                if (nbuf + rows > 32) {
+                    flush_rows(ws, G, w.split, brow0, nbuf, mine, lane);
+                    brow0 = row0;
+                    nbuf = 0;
+                }
+#pragma unroll
+                for (int r = 0; r < q4s::kRows; ++r)
+                    if (r < rows && lane == nbuf + r) mine = acc[r];
+                nbuf += rows;
             }
+            if (nbuf > 0) flush_rows(ws, G, w.split, brow0, nbuf, mine, lane);
             pos = p1;
         }
     }
