@@ -24,8 +24,9 @@
 //   producer warp         per stage, on one barrier: the codes (one 2-D TMA box,
 //                         128-byte swizzle), the activations (one box, binary32)
 //                         and the scales (one box, or one bulk copy per row)
-//   x warps (4)           activations -> bf16 hi/lo B operands (shared -> shared)
-//   dequant warps (4)     codes -> (q - 8) bf16 A operands in tensor memory
+//   operand warps (8)     activations -> bf16 hi/lo B operands (shared -> shared),
+//                         then codes -> (q - 8) bf16 A operands in tensor memory
+//                         (two warps per tensor-memory lane quarter)
 //   MMA issuers (2)       tcgen05.mma M = 128, N = 16 or 32, K = 16, one thread
 //                         each, quads alternating; per quad all blocks chunk by
 //                         chunk (consecutive MMAs accumulate into different
@@ -250,57 +251,20 @@ __device__ void run_producer(const Ctx& C, const q4t::Params& P, int lane) {
     __syncwarp();
 }
 
-// ---- x warps: activations (shared, binary32) -> hi/lo B operands ----
+// ---- operand warps: activations -> hi/lo B operands, codes -> A operands ----
+// Eight warps (two per tensor-memory lane quarter) per stage: first the
+// stage's activations (shared binary32 -> bf16 hi/lo, items split over the 256
+// threads), then quad by quad the (q - 8) bf16 A operands of their blocks (warp
+// half h takes the blocks of a quad with block % 2 == h).
 template <int BT>
-__device__ void run_x(const Ctx& C, const q4t::Params& P, int xw, int lane) {
+__device__ void run_prep(const Ctx& C, const q4t::Params& P, int warp, int lane) {
     constexpr int kN = q4t::mma_n(BT);
-    constexpr int kMaxItems = (BT * q4t::kS * 4 + 127) / 128;
-    const int tid = xw * 32 + lane;  // 0..127
-    pdl_wait();  // every stage barrier also waits for the activations
-    q4t::Walk wk;
-    wk.begin(C.lo, C.hi);
-    q4t::Stage s;
-    uint32_t q = 0;
-    while (!warp_aborted(C) && wk.next(P, &s)) {
-        const int st = (int)(q % q4t::kStages);
-        const uint32_t v = q / q4t::kStages;
-        if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;
-        const int c0 = s.kb0 - q4t::window_of(s.kb0);
-        const int per_t = s.nblk * 4;
-        const int items = P.b * per_t;
-        const uint8_t* raw = C.smem + q4t::stage_xraw(st);
-        uint8_t* xs = C.smem + q4t::stage_xop(st);
-#pragma unroll
-        for (int m = 0; m < kMaxItems; ++m) {
-            const int it = tid + 128 * m;
-            if (it < items) {
-                const int t = it / per_t, rem = it - t * per_t;
-                const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
-                const float4* src = reinterpret_cast<const float4*>(
-                    raw + t * (q4t::kS * 128) + (c0 + i) * 128 + c2 * 64 + hh * 32);
-                const float4 xa = src[0], xb = src[1];
-                const float e[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-                uint4 H, L;
-                q4tm::split_row(e, &H, &L);
-                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 0)) = H;
-                *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 1)) = L;
-            }
-        }
-        // the MMA reads these operands through the async proxy
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(C.bar(q4t::kBarXOpFull + st));
-            mbar_arrive(C.bar(q4t::kBarStageEmpty + st));
-        }
-        ++q;
-    }
-}
-
-// ---- dequant warps: codes -> (q - 8) bf16 in tensor memory, quad by quad ----
-__device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane) {
-    const int r = dw * 32 + lane;
-    const uint32_t tlane = C.tmem + ((uint32_t)(dw * 32) << 16);
+    constexpr int kThreadsX = q4t::kPrepWarps * 32;
+    constexpr int kMaxItems = (BT * q4t::kS * 4 + kThreadsX - 1) / kThreadsX;
+    const int quarter = warp & 3, half = warp >> 3;
+    const int r = quarter * 32 + lane;  // tensor-memory lane = tile row
+    const int tid = half * 128 + r;     // 0..255
+    const uint32_t tlane = C.tmem + ((uint32_t)(quarter * 32) << 16);
     pdl_wait();  // every stage barrier also waits for the activations
     q4t::Walk wk;
     wk.begin(C.lo, C.hi);
@@ -311,8 +275,36 @@ __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane
         const int st = (int)(q % q4t::kStages);
         const uint32_t v = q / q4t::kStages;
         if (!waitw(C, P, q4t::kBarFull + st, v & 1u)) break;
-        const uint8_t* codes = C.smem + q4t::stage_codes(st);
         const int c0 = s.kb0 - q4t::window_of(s.kb0);
+        // activations
+        {
+            const int per_t = s.nblk * 4;
+            const int items = P.b * per_t;
+            const uint8_t* raw = C.smem + q4t::stage_xraw(st);
+            uint8_t* xs = C.smem + q4t::stage_xop(st);
+#pragma unroll
+            for (int m = 0; m < kMaxItems; ++m) {
+                const int it = tid + kThreadsX * m;
+                if (it < items) {
+                    const int t = it / per_t, rem = it - t * per_t;
+                    const int i = rem >> 2, c2 = (rem >> 1) & 1, hh = rem & 1;
+                    const float4* src = reinterpret_cast<const float4*>(
+                        raw + t * (q4t::kS * 128) + (c0 + i) * 128 + c2 * 64 + hh * 32);
+                    const float4 xa = src[0], xb = src[1];
+                    const float e[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                    uint4 H, L;
+                    q4tm::split_row(e, &H, &L);
+                    *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 0)) = H;
+                    *reinterpret_cast<uint4*>(xs + q4t::x_row_off(kN, i, c2, hh, t, 1)) = L;
+                }
+            }
+            // the MMA reads these operands through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(C.bar(q4t::kBarXOpFull + st));
+        }
+        // A operands, quad by quad
+        const uint8_t* codes = C.smem + q4t::stage_codes(st);
         for (int i0 = 0; i0 < s.nblk; i0 += q4t::kQ, ++j) {
             const int sa = (int)(j % q4t::kRingA);
             const uint32_t ua = j / q4t::kRingA;
@@ -322,18 +314,19 @@ __device__ void run_dequant(const Ctx& C, const q4t::Params& P, int dw, int lane
             }
             tc_fence_after();
             const int nq = s.nblk - i0 < q4t::kQ ? s.nblk - i0 : q4t::kQ;
-            // the quad's code bytes first (one 16-byte load per block), then the
-            // blocks' operands
-            uint4 qv[q4t::kQ];
+            uint4 qv[q4t::kQ / 2];
 #pragma unroll
-            for (int ii = 0; ii < q4t::kQ; ++ii)
-                qv[ii] = ii < nq ? *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i0 + ii))
-                                 : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < q4t::kQ / 2; ++k) {
+                const int ii = 2 * k + half;
+                qv[k] = ii < nq ? *reinterpret_cast<const uint4*>(codes + q4t::code_off(r, c0 + i0 + ii))
+                                : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-            for (int ii = 0; ii < q4t::kQ; ++ii) {
+            for (int k = 0; k < q4t::kQ / 2; ++k) {
+                const int ii = 2 * k + half;
                 if (ii < nq) {
                     uint32_t a[16];
-                    q4tm::dequant_block(qv[ii], a);
+                    q4tm::dequant_block(qv[k], a);
                     tc_st16(tlane + q4t::a_col(sa, ii), a);
                 }
             }
@@ -591,12 +584,10 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
 
     pdl_launch_dependents();
 
-    if (warp < q4t::kEpiWarp0) {
-        run_dequant(C, P, warp - q4t::kDequantWarp0, lane);
-    } else if (warp < q4t::kXWarp0) {
+    if (warp < q4t::kEpiWarp0 || (warp >= q4t::kEpiWarp0 + 4 && warp < q4t::kProdWarp)) {
+        run_prep<BT>(C, P, warp, lane);
+    } else if (warp < q4t::kEpiWarp0 + 4) {
         run_epilogue<BT>(C, P, warp - q4t::kEpiWarp0, lane);
-    } else if (warp < q4t::kProdWarp) {
-        run_x<BT>(C, P, warp - q4t::kXWarp0, lane);
     } else if (warp == q4t::kProdWarp) {
         run_producer<BT>(C, P, lane);
     } else {

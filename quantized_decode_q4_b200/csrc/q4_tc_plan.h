@@ -71,10 +71,12 @@ constexpr int kStageBytes = kCodesBytes + kXRawBytes + kXOpBytes + kDBytes;
 constexpr int kHeaderBytes = 1024;  // barriers, tensor-memory address, abort flag
 constexpr int kSmemBytes = kHeaderBytes + kStages * kStageBytes;
 
-// warp roles
-constexpr int kDequantWarp0 = 0;  // 4 warps: codes -> (q - 8) bf16 into tensor memory
+// warp roles: warps 0-3 and 8-11 prepare the operands (two per tensor-memory lane
+// quarter: warp w reaches lanes 32 (w % 4) .. 32 (w % 4) + 31; the warps of half
+// w / 8 dequantise the blocks of a quad with block % 2 == w / 8, and all eight
+// share the stage's activations)
+constexpr int kPrepWarps = 8;
 constexpr int kEpiWarp0 = 4;      // 4 warps: accumulators x scale, partial sums, y
-constexpr int kXWarp0 = 8;        // 4 warps: xraw -> bf16 hi/lo B operands
 constexpr int kProdWarp = 12;     // TMA loads (lane 0) and per-row scale copies (all lanes)
 constexpr int kMmaWarp0 = 13;     // 2 warps, one thread each: tcgen05.mma issue, quads
                                   // alternating between them
@@ -110,10 +112,11 @@ constexpr int kAbortOff = kTmemAddrOff + 4;  // int32 abort flag
 static_assert(kAbortOff + 4 <= kHeaderBytes, "header");
 
 // arrivals per barrier phase
-constexpr uint32_t kArrivalsStageEmpty = 4 + 4 + 4 + kMmaIssuers;  // dequant, x, epilogue
-                                                                   // warps; MMA issuers
-constexpr uint32_t kArrivalsXOpFull = 4;
-constexpr uint32_t kArrivalsAFull = 4;
+constexpr uint32_t kArrivalsStageEmpty = kPrepWarps + 4 + kMmaIssuers;  // operand and
+                                                                       // epilogue warps,
+                                                                       // MMA issuers
+constexpr uint32_t kArrivalsXOpFull = kPrepWarps;
+constexpr uint32_t kArrivalsAFull = kPrepWarps;
 constexpr uint32_t kArrivalsDEmpty = 4;
 
 Q4T_HD uint32_t stage_base(int st) { return (uint32_t)(kHeaderBytes + st * kStageBytes); }
