@@ -88,18 +88,23 @@ struct XDigits {
 __host__ __device__ __forceinline__ float block_dot_int(const uint4 q, const XDigits& x, int32_t ca,
                                                         int32_t cb, int32_t cc) {
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-    int32_t A = ca, B = cb, C = cc;
+    // two chains per digit plane (low and high nibbles) halve the dependent
+    // dp4a chain length
+    int32_t A = ca, B = cb, C = cc, A2 = 0, B2 = 0, C2 = 0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         const uint32_t lo = words[w] & 0x0F0F0F0Fu;         // codes 4w .. 4w+3
         const uint32_t hi = (words[w] >> 4) & 0x0F0F0F0Fu;  // codes 16+4w .. 16+4w+3
         A = dp4a_us(lo, x.a[w], A);
-        A = dp4a_us(hi, x.a[w + 4], A);
+        A2 = dp4a_us(hi, x.a[w + 4], A2);
         B = dp4a_us(lo, x.b[w], B);
-        B = dp4a_us(hi, x.b[w + 4], B);
+        B2 = dp4a_us(hi, x.b[w + 4], B2);
         C = dp4a_us(lo, x.c[w], C);
-        C = dp4a_us(hi, x.c[w + 4], C);
+        C2 = dp4a_us(hi, x.c[w + 4], C2);
     }
+    A += A2;
+    B += B2;
+    C += C2;
     return fmaf((float)A, 65536.0f, fmaf((float)B, 256.0f, (float)C));
 }
 
