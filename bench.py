@@ -171,6 +171,23 @@ class OracleSample:
                 return reps, dt
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of every rank's value (all ranks must call it, in the same order)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: float, steps: int, ms_max: float) -> float:
+    """Whole-job weight GB/s: every rank streams bytes_per_step per step; the job takes the
+    slowest rank's time."""
+    return world * bytes_per_step * steps / (ms_max / 1e3) / 1e9
+
+
 def reference_arm(args, workload):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -270,12 +287,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # every rank holds its own replica of the decode step (independent requests)
     step = DecodeStep(workload, args.batch, dev)
@@ -313,7 +324,7 @@ def main():
     barrier()
     clock_info = clocks.stop()
     ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms_local)
+    ms = max_over_ranks(ms_local, world, dev)
     sec = ms / 1e3
 
     # end to end through the C ABI: per step, activations host -> device from pinned
@@ -337,11 +348,11 @@ def main():
         e1.record(stream)
     e1.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     q4_bytes = step.q4_bytes
-    value = world * q4_bytes * args.steps / sec / 1e9
-    e2e = world * q4_bytes * args.steps / (e2e_ms / 1e3) / 1e9
+    value = whole_job_gbs(world, q4_bytes, args.steps, ms)
+    e2e = whole_job_gbs(world, q4_bytes, args.steps, e2e_ms)
     peak, peak_src = hbm_peak()
     per_gpu_alg = step.algorithmic_bytes * args.steps / sec / 1e9
     traffic = recorded_traffic(args.workload, args.batch)
