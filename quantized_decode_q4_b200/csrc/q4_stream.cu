@@ -121,42 +121,67 @@ __device__ __forceinline__ void wait_stage(uint32_t* ws, uint64_t* bar, uint32_t
 }
 
 // Stage the activations of split `split` of GEMV `G` in 24-bit block fixed
-// point (all threads of the CTA). Warp w quantises blocks w, w + kWarps, ...;
-// lane l holds element l of the block. All loads are issued first; they read
-// L2 (the activations may have been written by another CTA of this launch).
+// point (all threads of the CTA). Eight lanes share a block: lane l of a warp
+// takes block (pass * 4 + l / 8) of the warp's blocks and its elements
+// 4 g .. 4 g + 3, g = l % 8 (one 16-byte load, from L2: the activations may have
+// been written by another CTA or kernel). The block's largest |x| and its digit
+// sums are reduced over the eight lanes with shuffles; each lane stores its four
+// elements' digits as one 32-bit word per digit plane (word g % 4 of entry
+// 2 p + g / 4), lane g = 0 the block constants.
 __device__ __forceinline__ void stage_x(const q4s::Desc& G, int split, uint4* xq, int warp,
                                         int lane) {
-    constexpr int kPer = (q4s::kMaxSplitBlocks + q4s::kWarps - 1) / q4s::kWarps;
+    constexpr int kBlocksPerWarp = (q4s::kMaxSplitBlocks + q4s::kWarps - 1) / q4s::kWarps;
+    constexpr int kPasses = (kBlocksPerWarp + 3) / 4;
     const int kbs = q4s::split_blocks(G, split);
     const float* xg = G.x + (int64_t)split * G.nb_split * 32;
-    float v[kPer];
+    const int g = lane & 7;
+    float4 v[kPasses];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const int j = warp + i * q4s::kWarps;
-        v[i] = j < kbs ? __ldcg(xg + j * 32 + lane) : 0.0f;
+    for (int p = 0; p < kPasses; ++p) {
+        // warp w quantises blocks w, w + kWarps, ... (four per pass)
+        const int j = warp + (p * 4 + (lane >> 3)) * q4s::kWarps;
+        v[p] = j < kbs ? __ldcg(reinterpret_cast<const float4*>(xg + j * 32 + 4 * g))
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
-    uint8_t* xb = reinterpret_cast<uint8_t*>(xq);
+    uint32_t* xw = reinterpret_cast<uint32_t*>(xq);
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const int j = warp + i * q4s::kWarps;
-        if (j < kbs) {
-            // |x| of non-negative binary32 values orders like their bit patterns
-            const float m = __uint_as_float(
-                __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[i]))));
+    for (int p = 0; p < kPasses; ++p) {
+        const int j = warp + (p * 4 + (lane >> 3)) * q4s::kWarps;
+        // |x| of non-negative binary32 values orders like their bit patterns
+        uint32_t m = max(max(__float_as_uint(fabsf(v[p].x)), __float_as_uint(fabsf(v[p].y))),
+                         max(__float_as_uint(fabsf(v[p].z)), __float_as_uint(fabsf(v[p].w))));
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float inv = q4dev::xq_inv(__uint_as_float(m));
+        const float e[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
+        uint32_t wa = 0, wb = 0, wc = 0;
+        int32_t sa = 0, sb = 0, sc = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
             int32_t a, b, c;
-            q4dev::x_digits(q4dev::xq_int(v[i], q4dev::xq_inv(m)), &a, &b, &c);
-            const int wi = lane >> 2, half = wi >> 2;
-            const int in16 = (wi & 3) * 4 + (lane & 3);
-            xb[q4s::xq_slot(j, 0 + half) * 16 + in16] = (uint8_t)a;
-            xb[q4s::xq_slot(j, 2 + half) * 16 + in16] = (uint8_t)b;
-            xb[q4s::xq_slot(j, 4 + half) * 16 + in16] = (uint8_t)c;
-            const int32_t sa = __reduce_add_sync(0xffffffffu, a);
-            const int32_t sb = __reduce_add_sync(0xffffffffu, b);
-            const int32_t sc = __reduce_add_sync(0xffffffffu, c);
-            if (lane == 0)
+            q4dev::x_digits(q4dev::xq_int(e[i], inv), &a, &b, &c);
+            wa |= ((uint32_t)a & 0xFFu) << (8 * i);
+            wb |= ((uint32_t)b & 0xFFu) << (8 * i);
+            wc |= ((uint32_t)c & 0xFFu) << (8 * i);
+            sa += a;
+            sb += b;
+            sc += c;
+        }
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) {
+            sa += __shfl_xor_sync(0xffffffffu, sa, off);
+            sb += __shfl_xor_sync(0xffffffffu, sb, off);
+            sc += __shfl_xor_sync(0xffffffffu, sc, off);
+        }
+        if (j < kbs) {
+            const int half = g >> 2, word = g & 3;
+            xw[q4s::xq_slot(j, 0 + half) * 4 + word] = wa;
+            xw[q4s::xq_slot(j, 2 + half) * 4 + word] = wb;
+            xw[q4s::xq_slot(j, 4 + half) * 4 + word] = wc;
+            if (g == 0)
                 xq[q4s::xq_slot(j, 6)] = make_uint4((uint32_t)(-8 * sa), (uint32_t)(-8 * sb),
                                                     (uint32_t)(-8 * sc),
-                                                    __float_as_uint(q4dev::xq_scale(m)));
+                                                    __float_as_uint(q4dev::xq_scale(__uint_as_float(m))));
         }
     }
 }
