@@ -182,9 +182,11 @@ q4_status plan_stream(const Shape* sh, int count, int64_t part_base, q4s::Params
         if (s != Q4_OK) return s;
         base_rows += sh[i].n * ceil_div(sh[i].k / Q4_QK, q4s::kMaxSplitBlocks);
     }
-    // enough rows for one full tile per warp of the grid, splitting K (in whole
-    // sub-steps of 32 blocks) when the matrices are short
-    const int64_t target = (int64_t)kNumSMs * Q4_STREAM_CTAS_PER_SM * q4s::kWarps * q4s::kRows;
+    // enough rows for one row per warp of the grid, splitting K (in whole
+    // sub-steps of 32 blocks) when the matrices are shorter (splitting further, to
+    // a full tile per warp, measured slower on the 8B-class stack: the split-K
+    // finish costs more than the idle lanes)
+    const int64_t target = (int64_t)kNumSMs * Q4_STREAM_CTAS_PER_SM * q4s::kWarps;
     const int64_t factor = base_rows >= target ? 1 : ceil_div(target, base_rows);
     int64_t rows = 0, tick = 0, part = part_base;
     for (int i = 0; i < count; ++i) {
