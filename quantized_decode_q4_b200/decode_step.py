@@ -67,8 +67,9 @@ class DecodeStep:
 
     @property
     def launches(self) -> int:
-        """Kernels one step launches: one per dependency group and 4-token chunk."""
-        return self.workload.n_groups * ((self.batch + 3) // 4)
+        """Kernels one step launches: one per dependency group (batch 1 on the CUDA
+        cores, 2..16 tokens on the tensor cores, all tokens in one launch)."""
+        return self.workload.n_groups
 
     def run(self, stream=None):
         q4.layer_stack(self.stack, self.batch, self.ws, stream)

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from parity_util import assert_gemv_close, oracle_rows, sample_rows
-from quantized_decode_q4_b200 import synth
+from quantized_decode_q4_b200 import q4, synth
 from quantized_decode_q4_b200.decode_step import DecodeStep
 
 pytestmark = pytest.mark.gpu
@@ -71,3 +71,15 @@ def test_8b_class_stack_full_size(b):
         step.run()
     torch.cuda.synchronize()
     check_step(step, 4, 200)
+
+
+@pytest.mark.parametrize("b", [1, 4])
+def test_step_launch_count(b):
+    """One kernel per dependency group, whatever the batch (the figure bench.py reports)."""
+    step = DecodeStep(synth.workloads()["smollm2_135m"], b)
+    step.run()
+    torch.cuda.synchronize()
+    c0 = q4.launch_count()
+    step.run()
+    torch.cuda.synchronize()
+    assert q4.launch_count() - c0 == step.launches == synth.workloads()["smollm2_135m"].n_groups
