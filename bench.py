@@ -170,6 +170,33 @@ class OracleSample:
             if dt >= seconds:
                 return reps, dt
 
+    def time_threads(self, seconds: float, threads: int):
+        """Passes of the sample completed by `threads` threads running it side by side
+        (the oracle's C calls release the GIL) within `seconds`."""
+        import threading
+        counts = [0] * threads
+        t0 = time.perf_counter()
+        deadline = t0 + seconds
+
+        def work(i):
+            while time.perf_counter() < deadline:
+                self.run_once()
+                counts[i] += 1
+
+        ts = [threading.Thread(target=work, args=(i,)) for i in range(threads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+        return sum(counts), time.perf_counter() - t0
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
 
 def max_over_ranks(v: float, world: int, device) -> float:
     """The largest of every rank's value (all ranks must call it, in the same order)."""
@@ -358,9 +385,13 @@ def main():
     traffic = recorded_traffic(args.workload, args.batch)
 
     if rank == 0:
+        # the oracle on the host: one thread, then every core of this process
         cpu = OracleSample(workload, args.batch)
-        reps, dt = cpu.time(args.cpu_seconds)
+        reps1, dt1 = cpu.time(args.cpu_seconds / 2)
+        cores = host_cores()
+        reps, dt = cpu.time_threads(args.cpu_seconds / 2, cores)
         cpu_gbs = cpu.q4_bytes * reps / dt / 1e9
+        cpu_gbs1 = cpu.q4_bytes * reps1 / dt1 / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -390,8 +421,12 @@ def main():
                          f"time; the step is {step.launches} launches of this one kernel, so "
                          "this equals bytes per launch / mean launch duration"),
             },
-            "cpu_baseline": {"value": cpu_gbs, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": cpu.desc + f", {reps} passes in {dt:.1f} s"},
+            "cpu_baseline": {"value": cpu_gbs, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": (cpu.desc.replace(", 1 thread", "") +
+                                        f", {cores} threads side by side: {reps} passes in "
+                                        f"{dt:.1f} s"),
+                             "single_thread": {"value": cpu_gbs1, "unit": UNIT, "cores": 1,
+                                               "passes": reps1, "seconds": round(dt1, 2)}},
             "e2e": {"value": e2e, "unit": UNIT,
                     "h2d_bytes_per_step": step.x_all.numel() * 4,
                     "d2h_bytes_per_step": step.y_all.numel() * 4},
