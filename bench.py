@@ -396,9 +396,14 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
+            "dtype": "f32" if args.batch == 1 else "bf16", "data": "synthetic",
             "config": {
                 "workload": args.workload, "batch": args.batch,
+                "arith": ("exact integer block dot products (4-bit codes x 24-bit block "
+                          "fixed-point activations, dp4a), binary32 scales and sums"
+                          if args.batch == 1 else
+                          "tcgen05 bf16 MMA: (q - 8) exact in bf16, activations as bf16 hi + lo "
+                          "(2^-16 relative), binary32 accumulators and sums"),
                 "gemvs_per_step": len(workload.gemvs), "q4_bytes_per_step": q4_bytes,
                 "weights": "Q4_0 planes (4.5 bits/weight), binary32 activations and sums",
                 "launch": ("one CUDA graph per step of PDL-chained group launches"
