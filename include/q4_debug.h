@@ -72,6 +72,18 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b);
  * operand layouts (up to 8 tokens, and 9..16). Returns the number of failures. */
 int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks);
 
+/* q4_gemv_batched (b = 1: the batch-1 kernel; b >= 2: the tensor-core kernel)
+ * with every stage barrier of the launch waiting for 16 bytes more than its
+ * copies bring, so that every bounded wait of the kernel runs out: a test of the
+ * timeout path without a GPU fault (all copies land; no wait is unbounded). The
+ * call returns like q4_gemv_batched; the kernel records Q4_ERR_TIMEOUT in the
+ * workspace header (read it with q4_workspace_status, clear it with
+ * q4_workspace_init), leaves its copies and MMAs complete and its tensor memory
+ * freed, and Y holds no meaningful values. Takes tens to hundreds of
+ * milliseconds (20 ms per wait that runs out). */
+q4_status q4_debug_gemv_stall(const q4_matrix* m, const float* X, int b, float* Y, void* ws,
+                              size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -174,6 +174,11 @@ def workspace(nbytes: int, device="cuda", stream=None) -> torch.Tensor:
     return ws
 
 
+def workspace_init(ws: torch.Tensor, stream=None) -> None:
+    """Zero a workspace again (clears a recorded timeout)."""
+    _check(lib().q4_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "q4_workspace_init")
+
+
 def workspace_status(ws: torch.Tensor, stream=None) -> int:
     return lib().q4_workspace_status(_ptr(ws), _stream(stream))
 

@@ -365,7 +365,7 @@ q4_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 // Enqueue one group (all token chunks) with partial sums from `part_base`. The
 // first launch may use PDL only if `pdl_first` is set.
 q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_t part_base,
-                       bool pdl_first, cudaStream_t stream) {
+                       bool pdl_first, cudaStream_t stream, uint32_t tx_extra = 0) {
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {calls[i].m.n, calls[i].m.k};
     if (b == 1) {
@@ -381,6 +381,7 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
             P.g[i].y = calls[i].y;
         }
         P.ws = static_cast<uint32_t*>(ws);
+        P.tx_extra = tx_extra;
         if (cuda_failed(q4k::launch_stream(P, grid, pdl_first, stream))) return Q4_ERR_CUDA;
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return Q4_OK;
@@ -401,6 +402,7 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
                 return Q4_ERR_CUDA;
         }
         P.ws = static_cast<uint32_t*>(ws);
+        P.tx_extra = tx_extra;
         if (cuda_failed(q4k::launch_tc(P, pdl_first, stream))) return Q4_ERR_CUDA;
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return Q4_OK;
@@ -1012,6 +1014,22 @@ int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count) {
         }
     }
     return 0;
+}
+
+q4_status q4_debug_gemv_stall(const q4_matrix* m, const float* X, int b, float* Y, void* ws,
+                              size_t ws_bytes, void* stream) {
+    if (!m) return Q4_ERR_INVALID_ARG;
+    GemvCall call = {*m, X, Y};
+    int64_t tickets = 0, part = 0;
+    q4_status s = check_group(&call, 1, b, &tickets, &part);
+    if (s != Q4_OK) return s;
+    if (b > 1 && b < kTcMinBatch) return Q4_ERR_UNSUPPORTED;  // CUDA-core batched kernel
+    const int64_t base = part_base_for(tickets);
+    if ((s = check_ws(ws, ws_bytes, (size_t)(base + part))) != Q4_OK) return s;
+    if ((s = ensure_device()) != Q4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = clear_tickets(ws, tickets, st)) != Q4_OK) return s;
+    return launch_group(&call, 1, b, ws, base, false, st, 16u);
 }
 
 int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b) {

@@ -48,6 +48,7 @@ struct OneGroup {
         return v;
     }
     __device__ uint32_t* ws() const { return P.ws; }
+    __device__ uint32_t tx_extra() const { return P.tx_extra; }
 };
 
 // Copy issuer of one warp: walks the warp's tiles in the same order as the math
@@ -94,7 +95,7 @@ struct Issuer {
         const q4s::LaneCopy c = q4s::lane_copy(G, wk.split, row0, rows, lane);
         const uint32_t bytes = c.active ? c.bytes : 0u;
         const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
-        if (lane == 0) mbar_arrive_expect_tx(bar, total);
+        if (lane == 0) mbar_arrive_expect_tx(bar, total + S.tx_extra());
         __syncwarp();
         if (c.active)
             bulk_g2s(stage_base + c.dst,
@@ -328,7 +329,9 @@ __device__ __forceinline__ void stream_body(const Src& S) {
                     }
                 }
                 __syncwarp();
-                if (!is.done()) {
+                // (under the stall test hook a stage's phase never completes, so it is
+                // never armed twice)
+                if (!is.done() && S.tx_extra() == 0) {
                     // the stage is free: refill it kStages tiles ahead (the proxy fence
                     // orders this warp's reads before the async writes)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

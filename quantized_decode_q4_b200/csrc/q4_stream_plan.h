@@ -75,7 +75,7 @@ struct Desc {
 struct Params {
     Desc g[Q4_MAX_GROUP];
     int32_t count;
-    int32_t pad_;
+    uint32_t tx_extra;  // 0; test hook: bytes every stage waits for beyond its copies
     int64_t total_rows;
     uint32_t* ws;
 };

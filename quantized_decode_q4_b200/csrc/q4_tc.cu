@@ -214,7 +214,7 @@ __device__ void run_producer(const Ctx& C, const q4t::Params& P, int lane) {
         }
         if (lane == 0) {
             mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(C.smem + 8 * (q4t::kBarFull + st)),
-                                  (uint32_t)q4t::kCodesBytes + kXBox + dbytes);
+                                  (uint32_t)q4t::kCodesBytes + kXBox + dbytes + P.tx_extra);
         }
         __syncwarp();
         if (lane == 0) {

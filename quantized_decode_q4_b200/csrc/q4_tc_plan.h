@@ -199,7 +199,7 @@ struct Params {
     int32_t b;      // tokens
     int64_t total;  // F, < 2^31
     int32_t grid;   // G
-    int32_t pad_;
+    uint32_t tx_extra;  // 0; test hook: bytes every stage waits for beyond its copies
     uint32_t* ws;
 };
 
