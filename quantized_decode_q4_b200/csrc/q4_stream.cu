@@ -245,21 +245,17 @@ __device__ __forceinline__ void stream_body(const Src& S) {
     for (int s = 0; s < q4s::kStages && !is.done(); ++s)
         is.issue(S, ring + s * q4s::kStageBytes, bars + s, lane);
 
-    // warm L2 with the activations of the first two pieces (a hint only: the
-    // reads that use them come after the wait on the previous kernel)
+    // warm L2 with the activations of the first piece (a hint only: the reads
+    // that use them come after the wait on the previous kernel)
     {
         const q4s::View v0 = S.view(0);
         int64_t lo0, hi0;
         q4s::cta_range(v0, blockIdx.x, gridDim.x, &lo0, &hi0);
-        if (lo0 < hi0 && warp < 2 && lane == 0) {
-            q4s::Where w0 = q4s::locate(v0, lo0);
-            const int64_t e0 = w0.seg_end < hi0 ? w0.seg_end : hi0;
-            if (warp == 0 || e0 < hi0) {
-                if (warp == 1) w0 = q4s::locate(v0, e0);
-                const q4s::Desc& G0 = v0.g[w0.g];
-                bulk_prefetch_l2(G0.x + (int64_t)w0.split * G0.nb_split * 32,
-                                 (uint32_t)q4s::split_blocks(G0, w0.split) * 128u);
-            }
+        if (lo0 < hi0 && warp == 0 && lane == 0) {
+            const q4s::Where w0 = q4s::locate(v0, lo0);
+            const q4s::Desc& G0 = v0.g[w0.g];
+            bulk_prefetch_l2(G0.x + (int64_t)w0.split * G0.nb_split * 32,
+                             (uint32_t)q4s::split_blocks(G0, w0.split) * 128u);
         }
     }
 
@@ -272,35 +268,17 @@ __device__ __forceinline__ void stream_body(const Src& S) {
         int64_t lo, hi;
         q4s::cta_range(V, blockIdx.x, gridDim.x, &lo, &hi);
         int64_t pos = lo;
-        // the activations of the first two pieces are staged together (one pair of
-        // CTA barriers); later pieces take turns with the two regions
-        {
-            const q4s::Where w0 = q4s::locate(V, pos);
-            const int64_t e0 = w0.seg_end < hi ? w0.seg_end : hi;
-            __syncthreads();  // every warp is done with earlier activations
-            if (pos < hi) stage_x(V.g[w0.g], w0.split, xq, warp, lane);
-            if (e0 < hi) {
-                const q4s::Where w1 = q4s::locate(V, e0);
-                stage_x(V.g[w1.g], w1.split, xq + q4s::kXBytes / 16, warp, lane);
-            }
-            __syncthreads();
-        }
-        int piece = 0;
         while (pos < hi) {
             const q4s::Where w = q4s::locate(V, pos);
             const int64_t p1 = w.seg_end < hi ? w.seg_end : hi;
             const int64_t seg_row0 = pos - w.row;
             const q4s::Desc& G = V.g[w.g];
-            uint4* xr = xq + (piece & 1) * (q4s::kXBytes / 16);
-            if (piece >= 2) {
-                __syncthreads();  // every warp is done with piece - 2, which used xr
-                stage_x(G, w.split, xr, warp, lane);
-                __syncthreads();
-            }
-            ++piece;
+            __syncthreads();  // every warp is done with the previous activations
+            stage_x(G, w.split, xq, warp, lane);
+            __syncthreads();
             const int kbs = q4s::split_blocks(G, w.split);
             const int nsub = (kbs + 31) >> 5;
-            const uint4* xl = xr + lane;
+            const uint4* xl = xq + lane;
             int64_t ra, rb;
             q4s::warp_rows(pos, p1, warp, &ra, &rb);
             // finished rows wait in the lanes (row brow0 + l in lane l) and are

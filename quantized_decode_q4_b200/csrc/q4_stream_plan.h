@@ -51,9 +51,8 @@ constexpr int kStageQs = kRows * kMaxSplitBlocks * 16;
 constexpr int kStageD = kRows * kDSlot * 2 + 32;
 constexpr int kStageBytes = kStageQs + kStageD;
 constexpr int kBarBytes = ((kWarps * kStages * 8 + 127) / 128) * 128;
-constexpr int kXBytes = kMaxSplitBlocks * 7 * 16;  // one piece's staged activations
-constexpr int kXRegions = 2;  // the first two pieces of a CTA are staged together
-constexpr int kSmemBytes = kBarBytes + kXRegions * kXBytes + kWarps * kStages * kStageBytes;
+constexpr int kXBytes = kMaxSplitBlocks * 7 * 16;
+constexpr int kSmemBytes = kBarBytes + kXBytes + kWarps * kStages * kStageBytes;
 
 static_assert(kStageBytes % 16 == 0, "stages must keep 16-byte alignment");
 static_assert(kMaxSplitBlocks % 32 == 0, "split size");
@@ -200,7 +199,7 @@ Q4S_HD void row_read_offsets(const Desc& G, int split, int64_t row0, int rows, i
 }
 
 Q4S_HD uint32_t stage_offset(int warp, int stage) {
-    return kBarBytes + kXRegions * kXBytes + (uint32_t)(warp * kStages + stage) * kStageBytes;
+    return kBarBytes + kXBytes + (uint32_t)(warp * kStages + stage) * kStageBytes;
 }
 
 // Staged activations, in 24-bit block fixed point: for block j of the split,
