@@ -25,11 +25,13 @@ extern "C" {
  * the number of the first failed check (see q4_api.cu). */
 int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b);
 
-/* The same replay for the persistent batch-1 streaming kernel: every CTA's unit
- * range, every warp's chunk sequence (the copy issuer's and the consumer's must
- * agree chunk for chunk), every bulk copy's source and stage slot, exactly-once
- * coverage of every (row, block), and split-K tickets and partial sums inside
- * their workspace regions. Returns 0 when every check holds. */
+/* The same replay for the persistent batch-1 streaming kernel: every CTA's row
+ * range (contiguous, non-empty, and inside one (GEMV, K split) segment whenever
+ * the grid has at least one CTA per segment), every warp's chunk sequence (the
+ * copy issuer's and the consumer's must agree chunk for chunk), every bulk
+ * copy's source and stage slot, exactly-once coverage of every (row, block), and
+ * split-K tickets and partial sums inside their workspace regions. Returns 0
+ * when every check holds. */
 int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count);
 
 /* Summary of the plan above: out[0] = CTAs (units), out[1] = dynamic shared

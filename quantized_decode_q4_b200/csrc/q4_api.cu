@@ -171,6 +171,47 @@ int64_t part_base_for(int64_t tickets) {
 // Streaming (batch 1) plan over `count` GEMVs: splits, units, grid, tickets and
 // partial sums laid out as for plan_shapes.
 constexpr int kNumSMs = 148;
+static_assert(kNumSMs * Q4_STREAM_CTAS_PER_SM <= q4s::kMaxGrid, "CTA range table too small");
+
+// CTA ranges of a streaming launch over the row space of P (segments already
+// laid out). With at least as many CTAs as segments, each segment gets whole
+// CTAs: one each, then one at a time to the segment whose CTAs carry the most
+// weight bytes (rows x blocks of the split), never more CTAs than rows; a
+// segment's rows are cut into equal ranges (to within one). A CTA then stages
+// one piece's activations, where a range across a segment boundary would stage
+// two and finish last. With more segments than CTAs the row space is cut into
+// `grid` equal ranges.
+void stream_cta_ranges(q4s::Params* P, int grid) {
+    struct Seg {
+        int64_t begin, rows, weight;
+        int ctas;
+    };
+    std::vector<Seg> seg;
+    for (int i = 0; i < P->count; ++i) {
+        const q4s::Desc& G = P->g[i];
+        for (int sp = 0; sp < G.splits; ++sp)
+            seg.push_back({G.row_begin + sp * G.n, G.n, G.n * q4s::split_blocks(G, sp), 1});
+    }
+    const int nseg = (int)seg.size();
+    if (nseg > grid) {
+        const uint64_t R = (uint64_t)P->total_rows;  // < 2^31
+        for (int c = 0; c <= grid; ++c) P->cta_lo[c] = (int32_t)(R * (uint32_t)c / (uint32_t)grid);
+        return;
+    }
+    // grid <= total rows, so a segment with a CTA to spare is always left
+    for (int left = grid - nseg; left > 0; --left) {
+        int best = -1;
+        for (int s = 0; s < nseg; ++s) {
+            if (seg[s].ctas >= seg[s].rows) continue;
+            if (best < 0 || seg[s].weight * seg[best].ctas > seg[best].weight * seg[s].ctas) best = s;
+        }
+        ++seg[best].ctas;
+    }
+    int c = 0;
+    for (const Seg& s : seg)
+        for (int j = 0; j < s.ctas; ++j) P->cta_lo[c++] = (int32_t)(s.begin + s.rows * j / s.ctas);
+    P->cta_lo[grid] = (int32_t)P->total_rows;
+}
 
 q4_status plan_stream(const Shape* sh, int count, int64_t part_base, q4s::Params* P, int* grid,
                       int64_t* tickets, int64_t* ws_end) {
@@ -216,6 +257,7 @@ q4_status plan_stream(const Shape* sh, int count, int64_t part_base, q4s::Params
     P->count = count;
     P->total_rows = rows;
     *grid = (int)std::min<int64_t>((int64_t)kNumSMs * Q4_STREAM_CTAS_PER_SM, rows);
+    stream_cta_ranges(P, *grid);
     *tickets = tick;
     *ws_end = part;
     return Q4_OK;
@@ -903,12 +945,16 @@ int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count) {
     };
     std::vector<std::vector<uint8_t>> cover(count);
     for (int i = 0; i < count; ++i) cover[i].assign((size_t)(sh[i].n * (sh[i].k / Q4_QK)), 0);
+    int64_t nseg = 0;
+    for (int i = 0; i < count; ++i) nseg += P.g[i].splits;
     int64_t prev_hi = 0;
     for (int cta = 0; cta < grid; ++cta) {
         int64_t lo, hi;
-        cta_range(P, cta, grid, &lo, &hi);
-        if (lo != prev_hi || hi < lo) return 6;
+        cta_range(P, cta, &lo, &hi);
+        if (lo != prev_hi || hi <= lo) return 6;
         prev_hi = hi;
+        // with a CTA per segment at least, no range crosses a segment boundary
+        if (nseg <= grid && locate(P, hi - 1).seg_end < hi) return 24;
         for (int warp = 0; warp < kWarps; ++warp) {
             // the math loop's order: pieces, this warp's rows, tiles
             std::vector<Tile> consumer;

@@ -43,6 +43,7 @@ struct OneGroup {
     __device__ q4s::View view(int) const {
         q4s::View v;
         v.g = P.g;
+        v.cta_lo = P.cta_lo;
         v.count = P.count;
         v.total_rows = P.total_rows;
         return v;
@@ -69,7 +70,7 @@ struct Issuer {
         for (; gi < ngroups; ++gi) {
             v = S.view(gi);
             int64_t lo, hi;
-            q4s::cta_range(v, blockIdx.x, gridDim.x, &lo, &hi);
+            q4s::cta_range(v, blockIdx.x, &lo, &hi);
             wk.begin(lo, hi, warp);
             has = wk.next_piece(v);
             if (has) {
@@ -250,7 +251,7 @@ __device__ __forceinline__ void stream_body(const Src& S) {
     {
         const q4s::View v0 = S.view(0);
         int64_t lo0, hi0;
-        q4s::cta_range(v0, blockIdx.x, gridDim.x, &lo0, &hi0);
+        q4s::cta_range(v0, blockIdx.x, &lo0, &hi0);
         if (lo0 < hi0 && warp == 0 && lane == 0) {
             const q4s::Where w0 = q4s::locate(v0, lo0);
             const q4s::Desc& G0 = v0.g[w0.g];
@@ -266,7 +267,7 @@ __device__ __forceinline__ void stream_body(const Src& S) {
     for (int gi = 0; gi < S.groups(); ++gi) {
         const q4s::View V = S.view(gi);
         int64_t lo, hi;
-        q4s::cta_range(V, blockIdx.x, gridDim.x, &lo, &hi);
+        q4s::cta_range(V, blockIdx.x, &lo, &hi);
         int64_t pos = lo;
         while (pos < hi) {
             const q4s::Where w = q4s::locate(V, pos);

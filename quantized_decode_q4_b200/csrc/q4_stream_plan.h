@@ -4,11 +4,14 @@
 // A launch covers one dependency group (up to Q4_MAX_GROUP GEMVs). Its work is
 // counted in rows of segments: segment (g, split) is K split `split` of every row
 // of GEMV g. Segments are ordered (g, split) and their rows laid end to end in
-// one "row space" of total_rows rows. CTA c of G owns rows
-// [R c / G, R (c + 1) / G) of that space; the part of its range inside one
+// one "row space" of total_rows rows. CTA c owns rows [cta_lo[c], cta_lo[c + 1])
+// of that space. The planner gives every segment whole CTAs when there are at
+// least as many CTAs as segments (so no CTA stages the activations of two
+// segments: such a CTA finishes last and the next launch waits for it), else
+// cuts the row space into equal ranges. The part of a CTA's range inside one
 // segment is a piece, and warp w of the CTA takes rows
-// [len w / W, len (w + 1) / W) of each piece, so every CTA and every warp gets
-// the same number of rows to within one. A warp walks its rows in tiles of up to
+// [len w / W, len (w + 1) / W) of each piece, so every warp of a CTA gets the
+// same number of rows to within one. A warp walks its rows in tiles of up to
 // kRows rows (x reuse) and streams each tile's code and scale bytes (every block
 // of the split) through a private ring of kStages shared-memory stages.
 #pragma once
@@ -45,6 +48,7 @@ constexpr int kWarps = Q4_STREAM_WARPS;        // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kRows = Q4_STREAM_ROWS;           // rows per tile (x reuse per warp)
 constexpr int kStages = Q4_STREAM_STAGES;       // ring depth per warp (one tile per stage)
+constexpr int kMaxGrid = 148 * Q4_STREAM_CTAS_PER_SM;  // B200 SMs x CTAs of a launch per SM
 constexpr int kMaxSplitBlocks = 128;            // K per split <= 4096
 constexpr int kDSlot = kMaxSplitBlocks + 16;    // uint16 per scale row (per-row copies)
 constexpr int kStageQs = kRows * kMaxSplitBlocks * 16;
@@ -78,11 +82,13 @@ struct Params {
     uint32_t tx_extra;  // 0; test hook: bytes every stage waits for beyond its copies
     int64_t total_rows;
     uint32_t* ws;
+    int32_t cta_lo[kMaxGrid + 1];  // CTA c owns rows [cta_lo[c], cta_lo[c + 1]) (< 2^31)
 };
 
 // One dependency group as the walks see it (Params has the same members).
 struct View {
     const Desc* g;
+    const int32_t* cta_lo;
     int32_t count;
     int64_t total_rows;
 };
@@ -117,10 +123,9 @@ Q4S_HD int split_blocks(const Desc& G, int split) {
 }
 
 template <class PV>
-Q4S_HD void cta_range(const PV& P, int cta, int grid, int64_t* lo, int64_t* hi) {
-    const uint64_t R = (uint64_t)P.total_rows;  // < 2^31
-    *lo = (int64_t)(R * (uint32_t)cta / (uint32_t)grid);
-    *hi = (int64_t)(R * (uint32_t)(cta + 1) / (uint32_t)grid);
+Q4S_HD void cta_range(const PV& P, int cta, int64_t* lo, int64_t* hi) {
+    *lo = P.cta_lo[cta];
+    *hi = P.cta_lo[cta + 1];
 }
 
 // Rows [*a, *b) of a piece [p0, p1) that warp w takes.

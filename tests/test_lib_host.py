@@ -133,6 +133,8 @@ def test_streaming_plans_replay_on_host():
         for shapes in {tuple(v) for v in groups.values()}:
             assert _check_stream(list(shapes)) == 0, shapes
     assert _check_stream([(5, 96), (700, 2080), (3, 4160)]) == 0
+    # more (GEMV, split) segments than CTAs: equal ranges across segment boundaries
+    assert _check_stream([(8, 65536)] * 8) == 0
 
 
 def _check_tc(shapes, b):
