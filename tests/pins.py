@@ -251,7 +251,10 @@ def check_gemv_exact(lib, cases: int = 40, seed: int = 11) -> None:
                             Fraction(0))
                 sabs = sum((abs(w_exact[r][i] * Fraction(float(X[t, i]))) for i in range(k)),
                            Fraction(0))
-                assert abs(float(Fraction(Y[t, r]) - exact)) <= (k - 1) * 2.0 ** -53 * float(sabs) * 1.01
+                tol = (k - 1) * 2.0 ** -53 * float(sabs) * 1.01
+                assert abs(float(Fraction(Y[t, r]) - exact)) <= tol, f"case {c} token {t} row {r}"
+                # each token's own sum of |w_hat x| (its tolerance term)
+                assert abs(float(Fraction(S[t, r]) - sabs)) <= tol, f"case {c} token {t} row {r}"
 
 
 ALL_CHECKS = (check_golden, check_dequant_exact, check_gemv_exact, check_fp16)

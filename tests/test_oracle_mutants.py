@@ -32,6 +32,10 @@ MUTANTS = {
     "high_nibble_weight": ("return j < 16 ? (byte & 0x0f) : (byte >> 4);",
                            "return j < 16 ? (byte >> 4) : (byte & 0x0f);"),
     "planes_swap": ("memcpy(qs + i * 16, blk + 2, 16);", "memcpy(qs + i * 16, blk + 1, 16);"),
+    # batched form (the pin's matrices have n < k, so these reads stay inside X)
+    "batched_token_zero": ("X + t * k, Y + t * n", "X, Y + t * n"),
+    "batched_x_stride": ("X + t * k, Y + t * n", "X + t * n, Y + t * n"),
+    "batched_abs_sum_row": ("abs_sum ? abs_sum + t * n : (double *)0", "abs_sum ? abs_sum : (double *)0"),
 }
 
 
