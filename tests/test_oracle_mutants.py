@@ -17,6 +17,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "q4_oracle.c")
 MUTANTS = {
     "scale_sign": ("m / -8.0f", "m / 8.0f"),
     "round_to_floor": ("scaled + 8.5f", "scaled + 8.0f"),
+    "divide_not_reciprocal": ("volatile float scaled = w[j] * id;",
+                              "volatile float scaled = (d != 0.0f) ? w[j] / d : 0.0f;"),
     "tie_last_index": ("if (a > amax) {", "if (a >= amax) {"),
     "nibble_order": ("(uint8_t)(q[j] | (q[j + ORACLE_QK / 2] << 4))",
                      "(uint8_t)((q[j] << 4) | q[j + ORACLE_QK / 2])"),
