@@ -137,6 +137,26 @@ def test_streaming_plans_replay_on_host():
     assert _check_stream([(8, 65536)] * 8) == 0
 
 
+def test_streaming_plans_replay_random_groups():
+    """Seeded random groups of 1..8 GEMVs (tiny to 14336-wide K, ragged rows): CTA ranges
+    inside one segment whenever the grid has a CTA per segment, equal ranges otherwise,
+    and every replay check of the test above."""
+    rng = np.random.default_rng(2024)
+    ns = [1, 2, 3, 5, 17, 31, 64, 100, 128, 147, 148, 149, 300, 1000, 2368, 4096, 5000]
+    kbs = [1, 2, 3, 7, 16, 31, 32, 33, 64, 100, 127, 128, 129, 200, 256, 448, 1000]
+    for _ in range(200):
+        shapes = [(int(rng.choice(ns)), 32 * int(rng.choice(kbs)))
+                  for _ in range(int(rng.integers(1, 9)))]
+        assert _check_stream(shapes) == 0, shapes
+    # narrow matrices with a very long K: more (GEMV, split) segments than CTAs,
+    # so the row space is cut into equal ranges across segment boundaries
+    rng = np.random.default_rng(7)
+    for _ in range(40):
+        shapes = [(int(rng.integers(1, 9)), 32 * int(rng.choice([1024, 1500, 2048, 4096])))
+                  for _ in range(int(rng.integers(3, 9)))]
+        assert _check_stream(shapes) == 0, shapes
+
+
 def _check_tc(shapes, b):
     L = q4.lib()
     f = L.q4_debug_check_tc
