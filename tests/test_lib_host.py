@@ -187,6 +187,19 @@ def test_tensor_core_plans_replay_on_host():
     assert _check_tc([(5, 96)], 1) != 0 and _check_tc([(5, 96)], 17) != 0
 
 
+def test_tensor_core_plans_replay_random_groups():
+    """Seeded random groups of 1..8 GEMVs (ragged 128-row tiles, block counts that are
+    and are not multiples of the 8-block window) for every token count 2..16."""
+    rng = np.random.default_rng(99)
+    ns = [1, 7, 127, 128, 129, 300, 1000, 4096, 5000]
+    kbs = [1, 3, 7, 8, 9, 18, 30, 44, 64, 100, 128, 129, 448]
+    for _ in range(60):
+        shapes = [(int(rng.choice(ns)), 32 * int(rng.choice(kbs)))
+                  for _ in range(int(rng.integers(1, 9)))]
+        b = int(rng.integers(2, 17))
+        assert _check_tc(shapes, b) == 0, (shapes, b)
+
+
 def test_tensor_core_operands_on_host():
     """The dequantised A operand is q - 8 exactly at every MMA position and an
     emulated MMA over the staged hi/lo activations gives the block sum."""
