@@ -84,3 +84,55 @@ def test_clock_sampler_parsing(tmp_path):
 def test_clock_sampler_without_nvidia_smi_reports_nothing():
     c = bench.Clocks(0)
     assert c.stop() is None
+
+
+def test_pack_dequant_timing_arithmetic(monkeypatch):
+    """time_pack_dequant on the CPU with stand-ins for the device pieces: 3 warm-up
+    and 10 timed calls of each, outputs reused, bytes 4nk + 9nk/16, GB/s and the
+    fraction of the given peak from the event time."""
+    import torch
+
+    from quantized_decode_q4_b200 import q4, synth
+
+    class Event:
+        def __init__(self, enable_timing=False):
+            self.t = None
+
+        def record(self, stream=None):
+            self.t = calls["n"]
+
+        def synchronize(self):
+            pass
+
+        def elapsed_time(self, end):
+            return 0.05 * (end.t - self.t)      # 50 us per call
+
+    calls = {"n": 0, "pack": 0, "dequant": 0}
+    real_empty = torch.empty
+
+    def fake_pack(w, out=None, stream=None):
+        calls["n"] += 1
+        calls["pack"] += 1
+        return out if out is not None else "planes"
+
+    def fake_dequant(m, out=None, stream=None):
+        calls["n"] += 1
+        calls["dequant"] += 1
+        assert m == "planes" and out is not None
+        return out
+
+    monkeypatch.setattr(torch.cuda, "Event", Event)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
+    monkeypatch.setattr(torch, "empty", lambda *a, **kw: real_empty(1))
+    monkeypatch.setattr(q4, "pack", fake_pack)
+    monkeypatch.setattr(q4, "dequant", fake_dequant)
+    monkeypatch.setattr(synth, "matrix", lambda *a, **kw: "w")
+    n, k = 14336, 4096
+    res = bench.time_pack_dequant(6548.5, n, k, reps=10)
+    assert calls["pack"] == 1 + 3 + 10 and calls["dequant"] == 3 + 10
+    nbytes = 4 * n * k + 9 * n * k // 16
+    assert res["bytes_per_call"] == nbytes
+    for name in ("pack", "dequant"):
+        assert abs(res[name]["us_per_call"] - 50.0) < 1e-9
+        assert abs(res[name]["gbs"] - nbytes / 50e-6 / 1e9) < 1e-6
+        assert abs(res[name]["frac"] - res[name]["gbs"] / 6548.5) < 1e-12
