@@ -198,6 +198,18 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def step_percentiles(ms: list) -> dict:
+    """Median, 10th and 90th percentile (linear interpolation) of single-step times."""
+    s = sorted(ms)
+
+    def q(p):
+        x = p * (len(s) - 1)
+        i = int(x)
+        return s[i] if i + 1 >= len(s) else s[i] + (s[i + 1] - s[i]) * (x - i)
+
+    return {"steps": len(s), "median_ms": q(0.5), "p10_ms": q(0.1), "p90_ms": q(0.9)}
+
+
 def max_over_ranks(v: float, world: int, device) -> float:
     """The largest of every rank's value (all ranks must call it, in the same order)."""
     if world == 1:
@@ -384,6 +396,20 @@ def main():
     ms = max_over_ranks(ms_local, world, dev)
     sec = ms / 1e3
 
+    # distribution of single steps (a separate pass: an event between steps keeps the
+    # next step's first launch from overlapping the previous step's last one)
+    try:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        with torch.cuda.stream(stream):
+            evs[0].record(stream)
+            for i in range(args.steps):
+                run_step()
+                evs[i + 1].record(stream)
+        evs[-1].synchronize()
+        step_dist = step_percentiles([evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)])
+    except Exception as e:  # reported, never allowed to lose the bench line
+        step_dist = {"error": f"{type(e).__name__}: {e}"}
+
     # end to end through the C ABI: per step, activations host -> device from pinned
     # memory, the step, and the results device -> host into pinned memory
     x_host = step.x_all.cpu().pin_memory()
@@ -473,6 +499,7 @@ def main():
             "gpu_launches": launches,
             "clocks": clock_info,
             "offline_kernels": offline,
+            "step_ms_single": step_dist,
         }
         print(json.dumps(line), flush=True)
     if graph is not None:

@@ -136,3 +136,14 @@ def test_pack_dequant_timing_arithmetic(monkeypatch):
         assert abs(res[name]["us_per_call"] - 50.0) < 1e-9
         assert abs(res[name]["gbs"] - nbytes / 50e-6 / 1e9) < 1e-6
         assert abs(res[name]["frac"] - res[name]["gbs"] / 6548.5) < 1e-12
+
+
+def test_step_percentiles_match_linear_interpolation():
+    import numpy as np
+    rng = np.random.default_rng(5)
+    for n in (1, 2, 3, 10, 200):
+        ms = list(rng.uniform(1.0, 2.0, n))
+        d = bench.step_percentiles(ms)
+        assert d["steps"] == n
+        for key, p in (("median_ms", 50), ("p10_ms", 10), ("p90_ms", 90)):
+            assert abs(d[key] - float(np.percentile(ms, p))) < 1e-12, (n, key)
