@@ -288,6 +288,79 @@ def time_pack_dequant(peak: float, n: int = 14336, k: int = 4096, reps: int = 10
     return res
 
 
+# Every configuration the workloads define beyond the headline one: (workload, batch).
+CONFIG_CASES = [("single_768", 1), ("gpt2_124m", 1), ("smollm2_360m", 1), ("smollm2_360m", 4),
+                ("minimind_26m", 1), ("minimind_26m", 2), ("minimind_26m", 8),
+                ("minimind_26m", 16), ("smollm2_135m", 1), ("smollm2_135m", 2),
+                ("smollm2_135m", 8), ("smollm2_135m", 16), ("llama8b_class", 4)]
+
+
+def measure_configs(peak: float, shared=None, min_steps: int = 200, max_seconds: float = 4.0) -> dict:
+    """Decode-step throughput of every configuration in CONFIG_CASES, L2-cold: R
+    byte-identical copies of the packed weights (R x weight bytes >= 4 x the 126 MB
+    L2) run in turn, all R steps captured in one CUDA graph; CUDA events on the
+    replaying stream around whole replays after 3 warm-up replays. Per configuration:
+    weight GB/s (Q4_0 bytes per step / step time), tokens/s (batch / step time), ms per
+    step and the roofline fraction of the algorithmic bytes (weights + x + y) against
+    the measured HBM peak. `shared` maps a workload name to a DecodeStep whose packed
+    weights are reused."""
+    import math
+
+    import torch
+
+    from quantized_decode_q4_b200 import q4, synth
+    from quantized_decode_q4_b200.decode_step import DecodeStep
+    out = {}
+    for name, b in CONFIG_CASES:
+        try:
+            wl = synth.workloads()[name]
+            base = (shared or {}).get(name)
+            step = DecodeStep(wl, b, mats=base.mats if base is not None else None)
+            r = max(1, math.ceil(4 * L2_BYTES / step.q4_bytes))
+            stacks = step.weight_copies(r)
+            stream = torch.cuda.Stream()
+            with torch.cuda.stream(stream):
+                for st in stacks:            # first use outside the capture
+                    q4.layer_stack(st, b, step.ws, stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for st in stacks:
+                    q4.layer_stack(st, b, step.ws, stream)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    g.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            one = e0.elapsed_time(e1) / 1e3
+            reps = max(1, min(math.ceil(min_steps / r), int(max_seconds / max(one, 1e-6))))
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            sec = e0.elapsed_time(e1) / 1e3 / (reps * r)
+            out[f"{name}_b{b}"] = {
+                "weight_gbs": step.q4_bytes / sec / 1e9, "tokens_per_s": b / sec,
+                "ms_per_step": sec * 1e3, "frac": step.algorithmic_bytes / sec / 1e9 / peak,
+                "q4_bytes_per_step": step.q4_bytes, "launches_per_step": step.launches,
+                "weight_copies": r, "steps_timed": reps * r,
+                "l2": f"cold: {r} weight copies, {r * step.q4_bytes / 1e6:.0f} MB in turn",
+                "kernel": "q4k::gemv_b1_kernel" if b == 1 else "q4k::gemv_tc_kernel"}
+            del g, stacks, step
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        except Exception as e:  # reported, never allowed to lose the bench line
+            out[f"{name}_b{b}"] = {"error": f"{type(e).__name__}: {e}"}
+    return out
+
+
 def profile_gemv(args):
     """Launches of a single GEMV (synthetic weights packed on the GPU) for profilers."""
     import torch
@@ -318,6 +391,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--launch", default="graph", choices=["graph", "direct"])
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration throughput table")
     ap.add_argument("--profile-gemv", metavar="N,K", default=None,
                     help="no bench line: run --warmup + --steps launches of one GEMV of this "
                          "shape for --batch tokens (a small case for ncu captures)")
@@ -446,6 +521,9 @@ def main():
             offline = time_pack_dequant(peak)
         except Exception as e:  # reported, never allowed to lose the bench line
             offline = {"error": f"{type(e).__name__}: {e}"}
+        # every other configuration, L2-cold (one GPU only: keeps scaling runs short)
+        configs = (measure_configs(peak, shared={args.workload: step}) if world == 1 and
+                   not args.no_configs else {"skipped": "measured at one GPU"})
         # the oracle on the host: one thread, then every core of this process
         cpu = OracleSample(workload, args.batch)
         reps1, dt1 = cpu.time(args.cpu_seconds / 2)
@@ -460,8 +538,10 @@ def main():
             "dtype": "f32" if args.batch == 1 else "bf16", "data": "synthetic",
             "config": {
                 "workload": args.workload, "batch": args.batch,
-                "arith": ("exact integer block dot products (4-bit codes x 24-bit block "
-                          "fixed-point activations, dp4a), binary32 scales and sums"
+                "arith": ("exact integer block dot products of 4-bit codes with 31-bit block "
+                          "fixed-point activations (two 16-bit digit planes, dp2a); a 1024-weight "
+                          "slice holding an element the fixed point cannot carry within 2^-14 "
+                          "of itself is multiplied in binary32; binary32 scales and sums"
                           if args.batch == 1 else
                           "tcgen05 bf16 MMA: (q - 8) exact in bf16, activations as bf16 hi + lo "
                           "(2^-16 relative), binary32 accumulators and sums"),
@@ -481,7 +561,7 @@ def main():
             "roofline": {
                 "bound": "hbm", "achieved": per_gpu_alg, "peak": peak, "unit": "GB/s",
                 "frac": per_gpu_alg / peak, "traffic": traffic,
-                "kernel": "q4k::gemv_stream_kernel" if args.batch == 1 else "q4k::gemv_tc_kernel",
+                "kernel": "q4k::gemv_b1_kernel" if args.batch == 1 else "q4k::gemv_tc_kernel",
                 "peak_source": peak_src,
                 "note": ("achieved = algorithmic bytes of a step (Q4_0 weights + x + y) / step "
                          f"time; the step is {step.launches} launches of this one kernel, so "
@@ -499,6 +579,7 @@ def main():
             "gpu_launches": launches,
             "clocks": clock_info,
             "offline_kernels": offline,
+            "configs": configs,
             "step_ms_single": step_dist,
         }
         print(json.dumps(line), flush=True)

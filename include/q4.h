@@ -160,16 +160,25 @@ q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, v
  * freed by this call.
  *   - A matrix whose scratch need, q4_workspace_bytes(n, k, 1), exceeds that size
  *     is rejected with Q4_ERR_WORKSPACE before anything is enqueued (every matrix
- *     of the 8B-class layer needs at most 82,176 bytes).
- *   - The first call on each device looks up the array's device address and
- *     configures the kernels for that device; make that first call before any
- *     stream capture.
+ *     of the 8B-class layer needs at most a few hundred bytes).
+ *   - The first call on each device configures the kernels for that device;
+ *     make that first call before any stream capture. The array's device
+ *     address is looked up on every call (with the device current).
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents; each call clears the tickets it uses before its kernel. Calls
  *     that overlap on the GPU (for instance on two streams) race on the array:
  *     serialise them.
+ *   - A bounded device wait that gives up is recorded in the array's status
+ *     header; q4_noalloc_status reports (and clears) it.
  * Errors: as q4_gemv. */
 q4_status q4_gemv_noalloc(const q4_matrix* m, const float* x, float* y, void* stream);
+
+/* q4_noalloc_status — Q4_ERR_TIMEOUT if a bounded device wait of any
+ * q4_gemv_noalloc call on the current device gave up since the last
+ * q4_noalloc_status, else Q4_OK; clears the record. Enqueued on `stream` after
+ * the calls it reports on, and synchronises that stream (call it off the hot
+ * path). The pages have no counterpart of this call. */
+q4_status q4_noalloc_status(void* stream);
 
 /* A decode step: `count` GEMVs in dependency groups. group[i] is the group of
  * GEMV i; groups are non-decreasing and run in order; the GEMVs of one group

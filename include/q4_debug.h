@@ -15,44 +15,42 @@
 extern "C" {
 #endif
 
-/* Plan one launch for `count` GEMVs (shapes n[i] x k[i], b tokens) exactly as the
- * library would, then replay every unit and warp of it on the host: each bulk
- * copy must stay inside its plane (the d plane counted with its 16-byte padding)
- * and inside its shared-memory slot, be 16-byte aligned and sized, the staged
- * activations must stay inside x and their shared-memory region, every
- * (row, block) must be covered exactly once, and split-K partials and tickets
- * must stay inside the workspace. Returns 0 when every check holds, otherwise
- * the number of the first failed check (see q4_api.cu). */
-int q4_debug_check_plan(const int64_t* n, const int64_t* k, int count, int b);
+/* Plan one batch-1 launch for `count` GEMVs (shapes n[i] x k[i]) exactly as the
+ * library would on a device with `num_sms` multiprocessors, then replay every
+ * piece and unit of it on the host: the shared-memory layout must fit the
+ * budget (two CTAs per SM) with every region aligned, every piece must stay
+ * inside its GEMV, its staged activations and per-(row, slice) partial sums
+ * inside their regions, every bulk copy must be 16-byte aligned and sized,
+ * inside its plane (the d plane counted with its 16-byte padding) and inside
+ * its slot, the scale each lane reads must be its own block's, every (row,
+ * slice) must be covered exactly once, and split-K tickets and partial sums
+ * must stay inside their workspace regions, disjoint between GEMVs. Returns 0
+ * when every check holds, otherwise the number of the first failed check (see
+ * q4_debug.cu). */
+int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms);
 
-/* The same replay for the persistent batch-1 streaming kernel: every CTA's row
- * range (contiguous, non-empty, and inside one (GEMV, K split) segment whenever
- * the grid has at least one CTA per segment), every warp's chunk sequence (the
- * copy issuer's and the consumer's must agree chunk for chunk), every bulk
- * copy's source and stage slot, exactly-once coverage of every (row, block), and
- * split-K tickets and partial sums inside their workspace regions. Returns 0
- * when every check holds. */
-int q4_debug_check_stream(const int64_t* n, const int64_t* k, int count);
-
-/* Summary of the plan above: out[0] = CTAs (units), out[1] = dynamic shared
- * memory bytes per CTA, out[2] = workspace bytes, out[3 + i] = K splits of GEMV i.
- * Returns Q4_OK or Q4_ERR_INVALID_ARG. */
+/* Summary of the batch-1 plan above for a 148-multiprocessor B200 (b must be 1):
+ * out[0] = CTAs (pieces), out[1] = dynamic shared memory bytes per CTA,
+ * out[2] = workspace bytes, out[3] = weight ring slots, out[4 + i] = K splits of
+ * GEMV i. Returns Q4_OK or Q4_ERR_INVALID_ARG. */
 q4_status q4_debug_plan_info(const int64_t* n, const int64_t* k, int count, int b, int64_t* out);
 
-/* Run the kernels' nibble unpack (compiled for the host from the same source) on
- * `count` pseudo-random code words from `seed` and on all words with one nonzero
- * nibble, comparing with plain nibble extraction. Returns the number of
- * mismatching values (0 when correct). */
+/* Run the binary32 path's nibble unpack (compiled for the host from the same
+ * source) on `count` pseudo-random code words from `seed` and on all words with
+ * one nonzero nibble, comparing with plain nibble extraction, and its block dot
+ * product on one-hot activations. Returns the number of mismatching values (0
+ * when correct). */
 int64_t q4_debug_check_unpack(uint64_t seed, int64_t count);
 
-/* Check the batch-1 kernel's integer block dot product on the host (the same
- * source compiled for the CPU): every |X| <= 8,355,711 splits into three digits
- * in -128..127 that add back up, and for `blocks` pseudo-random blocks of codes
- * and activations over many magnitudes (zeros, 1e-20, 1e30, one dominant
- * element) the block sum times its scale is within
- * sum_j |q_j - 8| (s/2 + |x_j| 2^-22) + 2^-22 |exact| of the exact sum; blocks
- * with max|x| < 1e-30 (taken as zero) within sum_j |q_j - 8| |x_j|. Returns
- * the number of failures (0 when correct). */
+/* Check the batch-1 kernel's activation quantisation and block dot products on
+ * the host (the same source compiled for the CPU): every |X| <= 2^30 sampled
+ * (boundaries and a stride) splits into two 16-bit digits that add back up; for
+ * `blocks` pseudo-random blocks of codes and activations (magnitudes from 2^-100
+ * to 2^99, single and paired outliers of 1e4..1e6, subnormal neighbours, exact
+ * zeros, all-zero blocks), an unflagged block's integer sum times its scale is
+ * within (2^-14 + 2^-23) sum_j |(q_j - 8) x_j| of the exact sum, a flagged
+ * block's binary32 sum within 33 * 2^-24 of it, and every block with an outlier
+ * is flagged. Returns the number of failures (0 when correct). */
 int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks);
 
 /* The same replay for the batched tensor-core kernel (2 <= b <= 16 tokens):
@@ -75,8 +73,8 @@ int q4_debug_check_tc(const int64_t* n, const int64_t* k, int count, int b);
 int64_t q4_debug_check_tc_operands(uint64_t seed, int64_t blocks);
 
 /* q4_gemv_batched (b = 1: the batch-1 kernel; b >= 2: the tensor-core kernel)
- * with every stage barrier of the launch waiting for 16 bytes more than its
- * copies bring, so that every bounded wait of the kernel runs out: a test of the
+ * with every stage (ring slot) barrier of the launch waiting for 16 bytes more
+ * than its copies bring, so that every bounded wait of the kernel runs out: a test of the
  * timeout path without a GPU fault (all copies land; no wait is unbounded). The
  * call returns like q4_gemv_batched; the kernel records Q4_ERR_TIMEOUT in the
  * workspace header (read it with q4_workspace_status, clear it with

@@ -76,7 +76,9 @@ def lib():
             "q4_status_string": ([c.c_int], c.c_char_p),
             "q4_launch_count": ([], c.c_uint64),
             "q4_last_cuda_error": ([], c.c_char_p),
-            "q4_debug_check_plan": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int], c.c_int),
+            "q4_debug_check_b1": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int], c.c_int),
+            "q4_gemv_noalloc": ([mp, vp, vp, vp], c.c_int),
+            "q4_noalloc_status": ([vp], c.c_int),
             "q4_debug_plan_info": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int,
                                     c.POINTER(i64)], c.c_int),
             "q4_debug_check_unpack": ([c.c_uint64, i64], i64),
@@ -283,6 +285,21 @@ def planes_to_blocks(qs: np.ndarray, d: np.ndarray, n: int, k: int) -> np.ndarra
     return out
 
 
+def gemv_noalloc(m: Q4Matrix, x: torch.Tensor, y: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """y = W x for one token with the library's fixed scratch array (no workspace)."""
+    y = y if y is not None else torch.empty(m.n, dtype=torch.float32, device=x.device)
+    cm = m.c()
+    _check(lib().q4_gemv_noalloc(ctypes.byref(cm), _ptr(x), _ptr(y), _stream(stream)),
+           "q4_gemv_noalloc")
+    return y
+
+
+def noalloc_status(stream=None) -> int:
+    """Q4_ERR_TIMEOUT (6) if a q4_gemv_noalloc wait gave up since the last call, else 0."""
+    return lib().q4_noalloc_status(_stream(stream))
+
+
 def launch_count() -> int:
     return lib().q4_launch_count()
 
@@ -291,19 +308,21 @@ def status_string(s: int) -> str:
     return lib().q4_status_string(s).decode()
 
 
-def check_plan(shapes, b: int = 1) -> int:
+def check_b1(shapes, num_sms: int = 148) -> int:
+    """Host replay of the batch-1 launch plan (0 when every check holds)."""
     n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
     k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
-    return lib().q4_debug_check_plan(n, k, len(shapes), b)
+    return lib().q4_debug_check_b1(n, k, len(shapes), num_sms)
 
 
-def plan_info(shapes, b: int = 1) -> dict:
+def plan_info(shapes) -> dict:
+    """The batch-1 plan of one launch on a 148-SM B200."""
     n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
     k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
-    out = (ctypes.c_int64 * (3 + len(shapes)))()
-    _check(lib().q4_debug_plan_info(n, k, len(shapes), b, out), "q4_debug_plan_info")
-    return {"units": out[0], "smem": out[1], "ws_bytes": out[2],
-            "splits": [out[3 + i] for i in range(len(shapes))]}
+    out = (ctypes.c_int64 * (4 + len(shapes)))()
+    _check(lib().q4_debug_plan_info(n, k, len(shapes), 1, out), "q4_debug_plan_info")
+    return {"pieces": out[0], "smem": out[1], "ws_bytes": out[2], "slots": out[3],
+            "splits": [out[4 + i] for i in range(len(shapes))]}
 
 
 def check_unpack(seed: int = 1, count: int = 100000) -> int:

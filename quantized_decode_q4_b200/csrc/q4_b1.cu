@@ -1,0 +1,360 @@
+// Batch-1 Q4_0 decode mat-vec for sm_100a.
+//
+// "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
+// section 3 "Dequantizzazione Integrata": the decode mat-vec dequantises in
+// registers; no dequantised weight is ever written to memory. The work split is
+// described in q4_b1_plan.h. Per CTA:
+//  * a producer warp streams the piece's units (8 rows x 32 blocks: 4 KB of codes
+//    and their binary16 scales) from HBM into a ring of shared-memory slots with
+//    bulk copies on the TMA engine, one full and one empty mbarrier per slot. It
+//    starts before the wait on the previous kernel (programmatic dependent
+//    launch): weights never depend on an earlier kernel, so consecutive launches
+//    overlap their weight streams;
+//  * eight consumer warps quantise the piece's activations once into shared
+//    memory (31-bit block fixed point as two 16-bit digit planes, q4_intdot.cuh),
+//    then take units round-robin. Lane l owns block l of the unit's slice: its
+//    activation digits stay in registers while the slice does not change, and
+//    for each of the unit's rows it reads the block's 16 code bytes with one
+//    128-bit shared load, forms sum_j (q_j - 8) X_j with 16 dp2a instructions,
+//    and applies the block's binary16 scale and power-of-two activation scale
+//    once. A slice holding a flagged block (an element the fixed point cannot
+//    carry within 2^-14 of itself) is multiplied in binary32 instead;
+//  * the 8 rows of a unit are summed over the lanes with shuffles and written to
+//    per-(row, slice) shared slots; after the last unit each row's slices are
+//    added in slice order (deterministic) and y is stored, or, for a K split
+//    across CTAs, a partial sum that the last split of the row to arrive adds up
+//    in split order.
+// Every wait is bounded (%globaltimer): a wait that gives up records
+// Q4_ERR_TIMEOUT in the workspace header and the CTA stops its work.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "q4_b1_plan.h"
+#include "q4_device.cuh"
+#include "q4_intdot.cuh"
+
+using namespace q4dev;
+
+namespace q4k {
+
+namespace {
+
+constexpr uint32_t kTimeoutFlag = 1u;
+constexpr int kConsumerBar = 1;  // named barrier of the consumer warps
+
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "n"(q4b::kConsumers * 32) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float half_bits_f32(uint32_t h) {
+    return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+// Quantise the piece's activations (all consumer threads): item i of
+// S * 32 * 8 is float4 g = i % 8 of block i / 8 (local slice (i / 8) / 32).
+// Eight consecutive lanes share a block; the block's largest |x|, digit sums and
+// flag are reduced over them with shuffles.
+__device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
+    const int items = S * q4b::kSliceBlocks * 8;
+    for (int base = 0; base < items; base += q4b::kConsumers * 32) {
+        const int i = base + tid;
+        const int jl = i >> 3, g = i & 7;
+        const int s = jl >> 5, jb = jl & 31;
+        const bool inside = i < items && jb < q4b::slice_blocks(G, s0 + s);
+        const int64_t b = (int64_t)(s0 + s) * q4b::kSliceBlocks + jb;
+        const float4 v = inside ? __ldcg(reinterpret_cast<const float4*>(G.x + b * 32) + g)
+                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        uint32_t m = max(max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu),
+                         max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu));
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float sc, inv;
+        bool ok = xq_scale(m, &sc, &inv);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        int32_t d0[4], d1[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            bool ek = true;
+            const int32_t X = ok ? xq_int(e[k], inv, &ek) : 0;
+            ok = ok && ek;
+            x_digits16(X, &d0[k], &d1[k]);
+        }
+        int32_t sum0 = d0[0] + d0[1] + d0[2] + d0[3], sum1 = d1[0] + d1[1] + d1[2] + d1[3];
+        uint32_t flag = ok ? 0u : 1u;
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) {
+            sum0 += __shfl_xor_sync(0xffffffffu, sum0, off);
+            sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
+            flag |= __shfl_xor_sync(0xffffffffu, flag, off);
+        }
+        if (i < items) {
+            const uint32_t half = (uint32_t)(g & 1) * 8u;
+            *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, g >> 1, jb) + half) =
+                make_uint2(pack16(d0[0], d0[1]), pack16(d0[2], d0[3]));
+            *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, 4 + (g >> 1), jb) + half) =
+                make_uint2(pack16(d1[0], d1[1]), pack16(d1[2], d1[3]));
+            if (g == 0)
+                *reinterpret_cast<uint4*>(xs + q4b::xchunk_offset(s, 8, jb)) =
+                    make_uint4((uint32_t)(-8 * sum0), (uint32_t)(-8 * sum1), __float_as_uint(sc), flag);
+        }
+    }
+}
+
+// Sum each of 8 rows over the 32 lanes: afterwards lane l holds the total of
+// row l / 4 (lanes 4r .. 4r + 3 all hold row r).
+__device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b4 ? v[i] : v[i + 4], keep = b4 ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b3 ? v[i] : v[i + 2], keep = b3 ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    {
+        const float send = b2 ? v[0] : v[1], keep = b2 ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+    return v[0];
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* ws,
+                                             volatile int* abort_flag, int lane) {
+    if (mbar_wait_bounded(bar, parity)) return true;
+    if (lane == 0) {
+        atomicOr(ws, kTimeoutFlag);
+        *abort_flag = 1;
+    }
+    return false;
+}
+
+// The producer warp: every unit of the piece, in order, into ring slot u % slots.
+__device__ __forceinline__ void produce(const q4b::Params& P, const q4b::Desc& G, const q4b::Piece& pc,
+                                        int s0, int S, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                        volatile int* abort_flag, int lane) {
+    const int T = q4b::piece_tiles(pc);
+    const int U = T * S;
+    const int slots = P.slots;
+    for (int u = 0; u < U; ++u) {
+        const int slot = u % slots, round = u / slots;
+        if (round > 0) {
+            const bool ok = wait_bounded(empty + slot, (uint32_t)(round - 1) & 1u, P.ws, abort_flag, lane);
+            if (!__all_sync(0xffffffffu, ok)) return;
+            // order the consumers' shared-memory reads of the slot before the copies
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        if (*abort_flag) return;
+        const int t = u / S, s = u - t * S;
+        const q4b::LaneCopy c = q4b::lane_copy(G, pc, t, s0 + s, lane);
+        const uint32_t bytes = c.active ? c.bytes : 0u;
+        const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+        if (lane == 0) mbar_arrive_expect_tx(full + slot, total + P.tx_extra);
+        __syncwarp();
+        if (c.active)
+            bulk_g2s(ring + (size_t)slot * q4b::kSlotBytes + c.dst,
+                     (c.scales ? reinterpret_cast<const uint8_t*>(G.d) : G.qs) + c.src_off, c.bytes,
+                     full + slot);
+    }
+}
+
+// Activation data of lane `lane` for local slice s.
+struct LaneX {
+    XPlanes p;
+    float scale;
+    bool flagged;  // some block of the slice takes the binary32 path
+};
+
+__device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, LaneX* lx) {
+    const uint32_t base = smem_addr(xs);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 a = lds128(base + q4b::xchunk_offset(s, q, lane));
+        const uint4 b = lds128(base + q4b::xchunk_offset(s, 4 + q, lane));
+        lx->p.a0[4 * q] = a.x;
+        lx->p.a0[4 * q + 1] = a.y;
+        lx->p.a0[4 * q + 2] = a.z;
+        lx->p.a0[4 * q + 3] = a.w;
+        lx->p.a1[4 * q] = b.x;
+        lx->p.a1[4 * q + 1] = b.y;
+        lx->p.a1[4 * q + 2] = b.z;
+        lx->p.a1[4 * q + 3] = b.w;
+    }
+    const uint4 k = lds128(base + q4b::xchunk_offset(s, 8, lane));
+    lx->p.c0 = (int32_t)k.x;
+    lx->p.c1 = (int32_t)k.y;
+    lx->scale = __uint_as_float(k.z);
+    lx->flagged = __any_sync(0xffffffffu, k.w != 0u);
+}
+
+}  // namespace
+
+__global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const q4b::Piece pc = q4b::piece_of(P, blockIdx.x);
+    const q4b::Desc& G = P.g[pc.g];
+    int s0, S;
+    q4b::piece_slices(G, pc.split, &s0, &S);
+    const int T = q4b::piece_tiles(pc);
+    const int U = T * S;
+    const int slots = P.slots;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + q4b::kMaxSlots;
+    float* red = reinterpret_cast<float*>(smem + q4b::red_offset());
+    uint8_t* xs = smem + q4b::x_offset(P);
+    uint8_t* ring = smem + q4b::ring_offset(P);
+    __shared__ int abort_flag;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < slots; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, 1);  // one consumer warp per use
+        }
+        abort_flag = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    if (warp == q4b::kConsumers) {
+        // weights never depend on an earlier kernel: stream before the wait
+        produce(P, G, pc, s0, S, ring, full, empty, &abort_flag, lane);
+        return;
+    }
+
+    pdl_wait();
+    const int tid = threadIdx.x;
+    stage_x(G, s0, S, xs, tid);
+    consumer_sync();
+
+    const uint32_t ring_base = smem_addr(ring);
+    int cur = -1;
+    LaneX lx;
+    volatile int* abort_v = &abort_flag;
+    for (int u = warp; u < U; u += q4b::kConsumers) {
+        if (*abort_v) break;
+        const int t = u / S, s = u - t * S;
+        if (s != cur) {
+            load_lane_x(xs, s, lane, &lx);
+            cur = s;
+        }
+        const int slot = u % slots;
+        const bool ok = wait_bounded(full + slot, (uint32_t)(u / slots) & 1u, P.ws, &abort_flag, lane);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int gs = s0 + s;
+        const int bs = q4b::slice_blocks(G, gs);
+        const int nr = min(q4b::kTileRows, pc.r1 - pc.r0 - t * q4b::kTileRows);
+        const uint32_t sb = ring_base + (uint32_t)slot * q4b::kSlotBytes;
+        float v[8];
+        if (!lx.flagged) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const uint4 q = lds128(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                const uint32_t dh = lds_u16(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
+                const float dot = block_dot16(q, lx.p);
+                v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * lx.scale * dot : 0.0f;
+            }
+        } else {
+            // exact path: binary32 products with the activations themselves
+            float4 xf[8];
+            const float4* xg = reinterpret_cast<const float4*>(G.x + ((int64_t)gs * q4b::kSliceBlocks + lane) * 32);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) xf[c] = lane < bs ? __ldcg(xg + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const UnpackConsts k = unpack_consts_default();
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const uint4 q = lds128(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                const uint32_t dh = lds_u16(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
+                const float2 d2 = block_dot(q, xf, k);
+                v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + slot);
+        const float row_sum = reduce8(v, lane);
+        const int r = lane >> 2;
+        if ((lane & 3) == 0 && r < nr) red[(t * q4b::kTileRows + r) * S + s] = row_sum;
+    }
+    consumer_sync();
+    if (*abort_v) return;
+
+    // each row's slices in slice order
+    const int rows = pc.r1 - pc.r0;
+    if (G.splits == 1) {
+        for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+            float sum = 0.0f;
+            for (int s = 0; s < S; ++s) sum += red[rl * S + s];
+            G.y[pc.r0 + rl] = sum;
+        }
+        return;
+    }
+    float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
+    uint32_t* tickets = P.ws + G.ticket_off;
+    for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+        float sum = 0.0f;
+        for (int s = 0; s < S; ++s) sum += red[rl * S + s];
+        part[(int64_t)pc.split * G.n + pc.r0 + rl] = sum;
+    }
+    __threadfence();
+    consumer_sync();
+    for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+        const int64_t row = pc.r0 + rl;
+        if (atomicAdd(tickets + row, 1u) == (uint32_t)G.splits - 1u) {
+            __threadfence();
+            float sum = 0.0f;
+            for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
+            G.y[row] = sum;
+            tickets[row] = 0u;
+        }
+    }
+}
+
+cudaError_t setup_b1_kernel(int optin_smem) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_b1_kernel);
+    if (e != cudaSuccess) return e;
+    if (q4b::kSmemBudget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
+    return cudaFuncSetAttribute(gemv_b1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                q4b::kSmemBudget);
+}
+
+cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P.npieces, 1, 1);
+    cfg.blockDim = dim3(q4b::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = q4b::smem_bytes(P);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_b1_kernel, P);
+}
+
+}  // namespace q4k

@@ -1,0 +1,175 @@
+// Work decomposition of the batch-1 decode mat-vec kernel, shared by the device
+// code and by the host replay in q4_debug_check_b1.
+//
+// A launch covers one dependency group (up to Q4_MAX_GROUP GEMVs). Its work is
+// cut into pieces, one per CTA: GEMV g owns pieces [piece_begin, piece_begin +
+// splits * cps), piece piece_begin + split * cps + j being rows
+// [n j / cps, n (j + 1) / cps) of K split `split` (K is split across CTAs for
+// narrow groups, whose rows are fewer than the CTAs of a launch, and for K beyond
+// 14 slices). Within a piece, K is walked in slices of 32
+// blocks (1024 weights, one block per lane) and rows in tiles of 8: unit
+// u = t * S + s is tile t, slice s of the piece's S slices (tile-major, so a
+// consumer warp that takes every 8th unit keeps one slice when S divides 8).
+//
+// Per CTA: one producer warp streams every unit's code bytes and binary16 scales
+// from HBM into a ring of shared-memory slots with bulk copies on the TMA
+// engine (one full and one empty mbarrier per slot); eight consumer warps take
+// units round-robin, multiply them with the piece's activations (quantised once
+// per piece into shared memory), and write per-(row, slice) partial sums to
+// shared memory; after the last unit the CTA adds each row's slices in slice
+// order and stores y (or a split-K partial, added up in split order by the last
+// split of the row to arrive). Two CTAs of consecutive launches fit one SM, so a
+// launch streams its weights in while the previous one finishes.
+#pragma once
+
+#include <cstdint>
+
+#include "../../include/q4.h"
+
+#if defined(__CUDACC__)
+#define Q4B_HD __host__ __device__ __forceinline__
+#else
+#define Q4B_HD inline
+#endif
+
+namespace q4b {
+
+constexpr int kConsumers = 8;                 // consumer warps
+constexpr int kWarps = kConsumers + 1;        // + the producer warp
+constexpr int kThreads = kWarps * 32;
+constexpr int kTileRows = 8;                  // rows per unit
+constexpr int kSliceBlocks = 32;              // blocks per unit (one per lane)
+constexpr int kSlotQs = kTileRows * kSliceBlocks * 16;  // code bytes of a unit
+constexpr int kDRow = 80;                     // scale bytes per row in a slot (64 + alignment slack)
+constexpr int kSlotBytes = kSlotQs + kTileRows * kDRow;
+constexpr int kXBlockBytes = 144;             // staged activation block: 32 digit words + 4 words
+constexpr int kXChunks = kXBlockBytes / 16;   // 16-byte chunks per staged block
+constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
+constexpr int kMaxSlots = 24;
+constexpr int kMinSlots = 6;
+constexpr int kBarBytes = 2 * kMaxSlots * 8;  // full[], empty[]
+// Shared memory of one CTA: two CTAs of consecutive launches share an SM.
+constexpr int kSmemBudget = 113 * 1024;
+
+static_assert(kSlotBytes % 128 == 0, "slots keep 128-byte alignment");
+static_assert(kXSliceBytes % 16 == 0, "staged slices keep 16-byte alignment");
+
+struct Desc {
+    const uint8_t* qs;
+    const uint16_t* d;
+    const float* x;
+    float* y;
+    int64_t n;
+    int32_t nb;                // k / 32
+    int32_t nslices;           // ceil(nb / 32)
+    int32_t splits;            // K splits across CTAs
+    int32_t slices_per_split;
+    int32_t piece_begin;       // first piece (CTA) of this GEMV
+    int32_t cps;               // pieces (CTAs) per split
+    int64_t part_off;          // floats: split-K partial sums [splits][n]
+    int64_t ticket_off;        // uint32: one ticket per row
+};
+
+struct Piece {
+    int32_t g, split;
+    int32_t r0, r1;            // rows of GEMV g (< 2^31)
+};
+
+struct Params {
+    Desc g[Q4_MAX_GROUP];
+    int32_t count;
+    int32_t slots;             // ring slots of this launch
+    uint32_t red_bytes;        // shared memory for per-(row, slice) partial sums
+    uint32_t x_bytes;          // shared memory for the staged activations
+    uint32_t tx_extra;         // 0; test hook: bytes every slot waits for beyond its copies
+    int32_t npieces;
+    uint32_t* ws;
+};
+
+// Piece c of a launch.
+template <class PP>
+Q4B_HD Piece piece_of(const PP& P, int c) {
+    int g = 0;
+    while (g + 1 < P.count && c >= P.g[g + 1].piece_begin) ++g;
+    const Desc& G = P.g[g];
+    const int local = c - G.piece_begin;
+    Piece p;
+    p.g = g;
+    p.split = local / G.cps;
+    const int j = local - p.split * G.cps;
+    p.r0 = (int32_t)(G.n * j / G.cps);
+    p.r1 = (int32_t)(G.n * (j + 1) / G.cps);
+    return p;
+}
+
+Q4B_HD uint32_t smem_bytes(const Params& P) {
+    return (uint32_t)kBarBytes + P.red_bytes + P.x_bytes + (uint32_t)P.slots * kSlotBytes;
+}
+Q4B_HD uint32_t red_offset() { return (uint32_t)kBarBytes; }
+Q4B_HD uint32_t x_offset(const Params& P) { return (uint32_t)kBarBytes + P.red_bytes; }
+Q4B_HD uint32_t ring_offset(const Params& P) { return (uint32_t)kBarBytes + P.red_bytes + P.x_bytes; }
+
+// Slices of a piece: first global slice and count.
+Q4B_HD void piece_slices(const Desc& G, int split, int* s0, int* S) {
+    *s0 = split * G.slices_per_split;
+    const int rest = G.nslices - *s0;
+    *S = rest < G.slices_per_split ? rest : G.slices_per_split;
+}
+
+// Blocks of global slice gs (32, or fewer in the last slice).
+Q4B_HD int slice_blocks(const Desc& G, int gs) {
+    const int rest = G.nb - gs * kSliceBlocks;
+    return rest < kSliceBlocks ? rest : kSliceBlocks;
+}
+
+Q4B_HD int piece_tiles(const Piece& p) { return (p.r1 - p.r0 + kTileRows - 1) / kTileRows; }
+
+// The copy lane `lane` of the producer issues for unit (tile t, local slice s)
+// of a piece: lanes 0..7 the code bytes of row r = lane, lanes 8..15 the
+// 16-byte aligned superset of that row's scales (the d plane is padded to 16
+// bytes, so a superset never leaves it).
+struct LaneCopy {
+    int64_t src_off;  // byte offset in the qs plane (code copy) or the d plane
+    uint32_t dst;     // byte offset inside a slot
+    uint32_t bytes;
+    bool active;
+    bool scales;
+};
+
+Q4B_HD LaneCopy lane_copy(const Desc& G, const Piece& p, int t, int gs, int lane) {
+    LaneCopy c;
+    const int r = lane & 7;
+    const int64_t row = (int64_t)p.r0 + (int64_t)t * kTileRows + r;
+    const int bs = slice_blocks(G, gs);
+    c.scales = lane >= 8;
+    c.active = lane < 16 && row < p.r1;
+    const int64_t e = row * G.nb + (int64_t)gs * kSliceBlocks;  // first block of the copy
+    if (!c.scales) {
+        c.src_off = e * 16;
+        c.dst = (uint32_t)(r * kSliceBlocks * 16);
+        c.bytes = (uint32_t)bs * 16u;
+    } else {
+        const int64_t a = e * 2, a0 = a & ~(int64_t)15;
+        c.src_off = a0;
+        c.dst = (uint32_t)(kSlotQs + r * kDRow);
+        c.bytes = (uint32_t)(((a + 2 * (int64_t)bs + 15) & ~(int64_t)15) - a0);
+    }
+    return c;
+}
+
+// Byte offset, inside a slot, of the scale of block `lane` of row r of the unit.
+Q4B_HD uint32_t scale_offset(const Desc& G, const Piece& p, int t, int gs, int r, int lane) {
+    const int64_t row = (int64_t)p.r0 + (int64_t)t * kTileRows + r;
+    const int64_t a = (row * G.nb + (int64_t)gs * kSliceBlocks) * 2;
+    return (uint32_t)(kSlotQs + r * kDRow + (int)(a & 15) + 2 * lane);
+}
+
+// Staged activation block j of local slice s: chunk q (0..8) of 16 bytes at
+// x_offset + ((s * 9 + q) * 32 + j) * 16, so that the 32 lanes of a warp read 32
+// consecutive chunks. Chunks 0-3: digit plane 0 words 0-15; chunks 4-7: plane 1;
+// chunk 8: (c0, c1, scale bits, flag).
+Q4B_HD uint32_t xchunk_offset(int s, int q, int j) {
+    return (uint32_t)(((s * kXChunks + q) * kSliceBlocks + j) * 16);
+}
+
+}  // namespace q4b

@@ -17,15 +17,6 @@ namespace q4dev {
 constexpr uint64_t kWaitLimitNs = 20ull * 1000 * 1000;
 // Longest a thread may sleep inside one try_wait before it re-checks the clock.
 constexpr uint32_t kSuspendHintNs = 100000;
-#ifndef Q4_WAIT_HINT
-#define Q4_WAIT_HINT 1
-#endif
-// Device unpack form: 2 = explicit PTX packing of each f32x2 pair (fewest
-// integer instructions); 0 = C++ pairs; 1 = scalar binary32. The host always
-// compiles form 0, which the host-side unpack check exercises.
-#ifndef Q4_UNPACK
-#define Q4_UNPACK 2
-#endif
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
@@ -58,21 +49,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 // false if it did not within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
     uint32_t done;
-#if Q4_WAIT_HINT
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(done)
         : "r"(addr), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
-#else
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-#endif
     return done != 0;
 }
 
@@ -187,11 +169,8 @@ __host__ __device__ __forceinline__ Pairs unpack_word(uint32_t q) {
     return p;
 }
 
-// Sum over one block of (q - 8) * x, with x given as 8 float4 chunks: chunk i
-// holds x[4i .. 4i+3] of the block. Returns two partial sums.
 // Constants of the register unpack: the magic exponents 2^23, 2^19, 2^15, 2^11,
-// 2^7 and the four (2^e + 8) offset pairs, as bit patterns. Kernels load them
-// once, from kernel parameters, so that they live in registers.
+// 2^7 and the four (2^e + 8) offset pairs, as bit patterns (held in registers).
 struct UnpackConsts {
     uint32_t e23, e19, e15, e11, e7;
     unsigned long long lo01, lo23, hi01, hi23;
@@ -211,33 +190,18 @@ __host__ __device__ __forceinline__ UnpackConsts unpack_consts_default() {
     return k;
 }
 
+// Sum over one block of (q - 8) * x, with x given as 8 float4 chunks (chunk i
+// holds x[4i .. 4i+3] of the block), as two partial sums: binary32 products of
+// the exact (q - 8) with x, two accumulator chains. On the device each pair is
+// packed from two logic results and handled by one f32x2 add and one f32x2
+// fused multiply-add; the host compiles the same arithmetic in C++ pairs (which
+// the host-side unpack check exercises).
 __host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4 (&x)[8],
                                                      const UnpackConsts& k) {
     float2 acc = f2(0.0f, 0.0f);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
     (void)k;
-#if Q4_UNPACK == 1 && !defined(__CUDA_ARCH__)
-#undef Q4_UNPACK
-#define Q4_UNPACK 0
-#endif
-#if Q4_UNPACK == 1
-    // scalar form: one logic op, one add and one fused multiply-add per weight
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const uint32_t v = words[w], sh = v >> 12;
-        acc.x = fmaf(__uint_as_float((v & 0xFu) | 0x4B000000u) - 8388616.0f, x[w].x, acc.x);
-        acc.y = fmaf(__uint_as_float((v & 0xF00u) | 0x47000000u) - 32776.0f, x[w].y, acc.y);
-        acc.x = fmaf(__uint_as_float((v & 0xF0000u) | 0x43000000u) - 136.0f, x[w].z, acc.x);
-        acc.y = fmaf(__uint_as_float((sh & 0xF000u) | 0x45000000u) - 2056.0f, x[w].w, acc.y);
-        acc.x = fmaf(__uint_as_float((v & 0xF0u) | 0x49000000u) - 524296.0f, x[w + 4].x, acc.x);
-        acc.y = fmaf(__uint_as_float((v & 0xF000u) | 0x45000000u) - 2056.0f, x[w + 4].y, acc.y);
-        acc.x = fmaf(__uint_as_float((sh & 0xF00u) | 0x47000000u) - 32776.0f, x[w + 4].z, acc.x);
-        acc.y = fmaf(__uint_as_float((sh & 0xF0000u) | 0x43000000u) - 136.0f, x[w + 4].w, acc.y);
-    }
-#elif Q4_UNPACK == 2 && defined(__CUDA_ARCH__)
-    // explicit PTX: each pair is packed from two logic results with mov.b64; two
-    // accumulator chains (even and odd words); the magic exponents and the pair
-    // offsets come in as registers
+#if defined(__CUDA_ARCH__)
     unsigned long long a[2] = {0ull, 0ull};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -283,12 +247,6 @@ __host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4
     }
 #endif
     return acc;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
 }
 
 }  // namespace q4dev

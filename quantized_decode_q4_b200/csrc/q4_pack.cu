@@ -60,43 +60,44 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w,
     }
 }
 
-// One thread per block: 16 code bytes and one scale -> 32 binary32 weights.
+// Eight threads per block, each writing four consecutive outputs as one 16-byte
+// store, so a warp writes 512 contiguous bytes (four blocks). Thread g of a block
+// writes outputs 4g .. 4g+3: for g < 4 these are the low nibbles of code word g,
+// for g >= 4 the high nibbles of code word g - 4 (byte m of a word carries
+// output 4w+m in its low nibble and output 16+4w+m in its high nibble).
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ qs,
                                                       const uint16_t* __restrict__ d,
                                                       float* __restrict__ out, int64_t nblocks) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nblocks; i += stride) {
-        const uint4 q = reinterpret_cast<const uint4*>(qs)[i];
+    const int64_t total = nblocks * 8;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += stride) {
+        const int64_t i = t >> 3;
+        const int g = (int)(t & 7);
+        const uint32_t word = reinterpret_cast<const uint32_t*>(qs)[i * 4 + (g & 3)];
+        const uint32_t nib = g < 4 ? word : word >> 4;
         const float s = __half2float(__ushort_as_half(d[i]));
-        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-        float v[32];
+        float v[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint32_t byte = (words[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-            v[j] = __fmul_rn(s, (float)((int)(byte & 0xFu) - 8));
-            v[j + 16] = __fmul_rn(s, (float)((int)(byte >> 4) - 8));
-        }
-        float4* dst = reinterpret_cast<float4*>(out) + i * 8;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        for (int m = 0; m < 4; ++m) v[m] = __fmul_rn(s, (float)((int)((nib >> (8 * m)) & 0xFu) - 8));
+        reinterpret_cast<float4*>(out)[t] = make_float4(v[0], v[1], v[2], v[3]);
     }
 }
 
-cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblocks,
+// Grids of at most 64 CTAs of 256 threads per multiprocessor (grid-stride loops).
+cudaError_t launch_pack(const float* w, uint8_t* qs, uint16_t* d, int64_t nblocks, int num_sms,
                         cudaStream_t stream) {
     const int threads = 256;
     int64_t blocks = (nblocks + threads - 1) / threads;
-    if (blocks > 148 * 64) blocks = 148 * 64;
+    if (blocks > (int64_t)num_sms * 64) blocks = (int64_t)num_sms * 64;
     pack_kernel<<<(unsigned)blocks, threads, 0, stream>>>(w, qs, d, nblocks);
     return cudaGetLastError();
 }
 
 cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int64_t nblocks,
-                           cudaStream_t stream) {
+                           int num_sms, cudaStream_t stream) {
     const int threads = 256;
-    int64_t blocks = (nblocks + threads - 1) / threads;
-    if (blocks > 148 * 64) blocks = 148 * 64;
+    int64_t blocks = (nblocks * 8 + threads - 1) / threads;
+    if (blocks > (int64_t)num_sms * 64) blocks = (int64_t)num_sms * 64;
     dequant_kernel<<<(unsigned)blocks, threads, 0, stream>>>(qs, d, out, nblocks);
     return cudaGetLastError();
 }

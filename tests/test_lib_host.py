@@ -87,74 +87,63 @@ EDGE_SHAPES = [(1, 32), (17, 32), (1, 96), (5, 64), (33, 4128), (3, 28672), (502
                (16, 4096), (15, 4096), (2, 131072)]
 
 
-@pytest.mark.parametrize("b", [1, 2, 3, 4])
-def test_launch_plans_replay_on_host(b):
-    for s in _all_shapes() + EDGE_SHAPES:
-        assert q4.check_plan([s], b) == 0, (s, b)
+def _groups_of_workloads():
+    out = set()
     for wl in synth.workloads().values():
         groups = {}
         for g in wl.gemvs:
             groups.setdefault(g.group, []).append((g.n, g.k))
-        for shapes in {tuple(v) for v in groups.values()}:
-            assert q4.check_plan(list(shapes), b) == 0, (shapes, b)
+        out |= {tuple(v) for v in groups.values()}
+    return sorted(out)
 
 
-def test_plan_properties():
-    info = q4.plan_info([(14336, 4096), (14336, 4096)], 1)
-    assert info["splits"] == [1, 1] and info["units"] == 1792 and info["ws_bytes"] == 256
-    assert info["smem"] <= 227 * 1024 // 4   # four CTAs fit on an SM
-    down = q4.plan_info([(4096, 14336)], 1)
-    assert down["splits"][0] >= 4            # K = 14336 does not fit one split
+@pytest.mark.parametrize("num_sms", [148, 132, 160, 7])
+def test_batch1_plans_replay_on_host(num_sms):
+    """Every byte the batch-1 kernel reads was copied from the right place and its
+    lane reads the scale of its own block, every (row, slice) is covered once, the
+    shared-memory layout fits two CTAs per SM, split-K scratch stays inside the
+    workspace - for every workload shape and group, the edge shapes, and devices
+    with other multiprocessor counts."""
+    for s in _all_shapes() + EDGE_SHAPES + [(1000, 2080), (3, 992), (4096, 14368)]:
+        assert q4.check_b1([s], num_sms) == 0, (s, num_sms)
+    for shapes in _groups_of_workloads():
+        assert q4.check_b1(list(shapes), num_sms) == 0, (shapes, num_sms)
+    assert q4.check_b1([(5, 96), (700, 2080), (3, 4160)], num_sms) == 0
+    assert q4.check_b1([(8, 65536)] * 8, num_sms) == 0
 
 
-def test_register_unpack_on_host():
-    assert q4.check_unpack(12345, 500000) == 0
-
-
-def _check_stream(shapes):
-    L = q4.lib()
-    f = L.q4_debug_check_stream
-    f.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
-    f.restype = ctypes.c_int
-    n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
-    k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
-    return f(n, k, len(shapes))
-
-
-def test_streaming_plans_replay_on_host():
-    """Every byte the batch-1 kernel reads was copied from the right place, every
-    (row, block) is covered once, copy issuer and math loop walk the same tiles."""
-    for s in _all_shapes() + EDGE_SHAPES + [(1000, 2080), (3, 992)]:
-        assert _check_stream([s]) == 0, s
-    for wl in synth.workloads().values():
-        groups = {}
-        for g in wl.gemvs:
-            groups.setdefault(g.group, []).append((g.n, g.k))
-        for shapes in {tuple(v) for v in groups.values()}:
-            assert _check_stream(list(shapes)) == 0, shapes
-    assert _check_stream([(5, 96), (700, 2080), (3, 4160)]) == 0
-    # more (GEMV, split) segments than CTAs: equal ranges across segment boundaries
-    assert _check_stream([(8, 65536)] * 8) == 0
-
-
-def test_streaming_plans_replay_random_groups():
-    """Seeded random groups of 1..8 GEMVs (tiny to 14336-wide K, ragged rows): CTA ranges
-    inside one segment whenever the grid has a CTA per segment, equal ranges otherwise,
-    and every replay check of the test above."""
+def test_batch1_plans_replay_random_groups():
+    """Seeded random groups of 1..8 GEMVs (tiny to 32768-wide K, ragged rows and
+    slices), including narrow groups whose K is split across CTAs."""
     rng = np.random.default_rng(2024)
     ns = [1, 2, 3, 5, 17, 31, 64, 100, 128, 147, 148, 149, 300, 1000, 2368, 4096, 5000]
-    kbs = [1, 2, 3, 7, 16, 31, 32, 33, 64, 100, 127, 128, 129, 200, 256, 448, 1000]
+    kbs = [1, 2, 3, 7, 16, 31, 32, 33, 64, 100, 127, 128, 129, 200, 256, 448, 449, 1000]
     for _ in range(200):
         shapes = [(int(rng.choice(ns)), 32 * int(rng.choice(kbs)))
                   for _ in range(int(rng.integers(1, 9)))]
-        assert _check_stream(shapes) == 0, shapes
-    # narrow matrices with a very long K: more (GEMV, split) segments than CTAs,
-    # so the row space is cut into equal ranges across segment boundaries
+        assert q4.check_b1(shapes) == 0, shapes
     rng = np.random.default_rng(7)
     for _ in range(40):
         shapes = [(int(rng.integers(1, 9)), 32 * int(rng.choice([1024, 1500, 2048, 4096])))
                   for _ in range(int(rng.integers(3, 9)))]
-        assert _check_stream(shapes) == 0, shapes
+        assert q4.check_b1(shapes) == 0, shapes
+
+
+def test_batch1_plan_properties():
+    gate_up = q4.plan_info([(14336, 4096), (14336, 4096)])
+    # no K split, one piece per multiprocessor, no split-K scratch
+    assert gate_up["splits"] == [1, 1] and gate_up["pieces"] == 148
+    assert gate_up["ws_bytes"] == 256
+    assert gate_up["smem"] <= 113 * 1024          # two CTAs share an SM
+    assert gate_up["slots"] >= 16                  # a deep weight ring
+    down = q4.plan_info([(4096, 14336)])
+    assert down["splits"] == [1] and down["slots"] >= 8
+    narrow = q4.plan_info([(2, 131072)])          # fewer rows than CTAs: K split
+    assert narrow["splits"][0] > 1 and narrow["ws_bytes"] > 256
+
+
+def test_register_unpack_on_host():
+    assert q4.check_unpack(12345, 500000) == 0
 
 
 def _check_tc(shapes, b):
@@ -211,7 +200,9 @@ def test_tensor_core_operands_on_host():
 
 
 def test_integer_block_dot_on_host():
-    """Activation digits split exactly; block sums within the stated bound."""
+    """Activation digits split exactly; unflagged block sums within 2^-14 of each
+    element, flagged blocks (outliers, subnormal neighbours, extreme ranges) on
+    the binary32 path within its rounding."""
     L = q4.lib()
     f = L.q4_debug_check_intdot
     f.argtypes = [ctypes.c_uint64, ctypes.c_int64]
