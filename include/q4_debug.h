@@ -20,13 +20,14 @@ extern "C" {
  * piece and unit of it on the host: the shared-memory layout must fit the
  * budget (two CTAs per SM) with every region aligned, every piece must stay
  * inside its GEMV, its staged activations and per-(row, slice) partial sums
- * inside their regions, every bulk copy must be 16-byte aligned and sized,
- * inside its plane (the d plane counted with its 16-byte padding) and inside
- * its slot, the scale each lane reads must be its own block's, every (row,
- * slice) must be covered exactly once, and split-K tickets and partial sums
- * must stay inside their workspace regions, disjoint between GEMVs. Returns 0
- * when every check holds, otherwise the number of the first failed check (see
- * q4_debug.cu). */
+ * inside their regions, every tensor-map box must start at a 16-byte aligned
+ * x coordinate inside its plane, every per-row scale copy (planes whose row
+ * stride is not a multiple of 16 bytes) must be 16-byte aligned and sized,
+ * inside the padded d plane and inside its slot, the scale each lane reads must
+ * be its own block's, every (row, slice) must be covered exactly once, and
+ * split-K tickets and partial sums must stay inside their workspace regions,
+ * disjoint between GEMVs. Returns 0 when every check holds, otherwise the number
+ * of the first failed check (see q4_debug.cu). */
 int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms);
 
 /* Summary of the batch-1 plan above for a 148-multiprocessor B200 (b must be 1):

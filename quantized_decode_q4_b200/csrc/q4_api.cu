@@ -92,6 +92,7 @@ q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4
         G.nslices = (int32_t)nsl;
         G.splits = (int32_t)splits;
         G.slices_per_split = (int32_t)sps;
+        G.d_map = nb % 8 == 0 ? 1 : 0;
         if (splits > 1) {
             G.ticket_off = kHeaderBytes / 4 + tick;
             tick += sh[i].n;
@@ -136,7 +137,8 @@ q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4
     P->red_bytes = (uint32_t)round_up(red_floats * 4, 128);
     P->x_bytes = (uint32_t)(max_slices * q4b::kXSliceBytes);
     const int64_t room = (int64_t)q4b::kSmemBudget - q4b::kBarBytes - P->red_bytes - P->x_bytes;
-    const int64_t slots = std::min<int64_t>(room / q4b::kSlotBytes, q4b::kMaxSlots);
+    // a multiple of the CTA's warps: each slot is requested and read by one warp
+    const int64_t slots = std::min<int64_t>(room / q4b::kSlotBytes, q4b::kMaxSlots) / q4b::kWarps * q4b::kWarps;
     if (slots < q4b::kMinSlots) return Q4_ERR_UNSUPPORTED;
     P->slots = (int32_t)slots;
     *tickets = tick;
@@ -317,6 +319,9 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
             P.g[i].d = calls[i].m.d;
             P.g[i].x = calls[i].x;
             P.g[i].y = calls[i].y;
+            if (cuda_failed(q4k::encode_b1_maps(&P.qs_map[i], &P.d_map[i], &P.g[i].d_map, calls[i].m.qs,
+                                                calls[i].m.d, calls[i].m.n, calls[i].m.k)))
+                return Q4_ERR_CUDA;
         }
         P.ws = static_cast<uint32_t*>(ws);
         P.tx_extra = tx_extra;

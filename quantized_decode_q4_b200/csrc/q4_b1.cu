@@ -3,22 +3,24 @@
 // "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
 // section 3 "Dequantizzazione Integrata": the decode mat-vec dequantises in
 // registers; no dequantised weight is ever written to memory. The work split is
-// described in q4_b1_plan.h. Per CTA:
-//  * a producer warp streams the piece's units (8 rows x 32 blocks: 4 KB of codes
-//    and their binary16 scales) from HBM into a ring of shared-memory slots with
-//    bulk copies on the TMA engine, one full and one empty mbarrier per slot. It
-//    starts before the wait on the previous kernel (programmatic dependent
-//    launch): weights never depend on an earlier kernel, so consecutive launches
-//    overlap their weight streams;
-//  * eight consumer warps quantise the piece's activations once into shared
-//    memory (31-bit block fixed point as two 16-bit digit planes, q4_intdot.cuh),
-//    then take units round-robin. Lane l owns block l of the unit's slice: its
-//    activation digits stay in registers while the slice does not change, and
-//    for each of the unit's rows it reads the block's 16 code bytes with one
-//    128-bit shared load, forms sum_j (q_j - 8) X_j with 16 dp2a instructions,
-//    and applies the block's binary16 scale and power-of-two activation scale
-//    once. A slice holding a flagged block (an element the fixed point cannot
-//    carry within 2^-14 of itself) is multiplied in binary32 instead;
+// described in q4_b1_plan.h. Per CTA (8 warps, two CTAs per SM):
+//  * the piece's units (8 rows x 32 blocks: 4 KB of codes and their binary16
+//    scales) stream from HBM into a ring of shared-memory slots as 2-D tensor
+//    loads on the TMA engine, each completing on its slot's mbarrier. The first
+//    units are requested before the wait on the previous kernel (programmatic
+//    dependent launch): weights never depend on an earlier kernel, so
+//    consecutive launches overlap their weight streams. A warp that has read a
+//    unit requests the unit `slots` further into the slot it just freed; the
+//    issuing lane rotates with the unit, so no thread has many copies in flight;
+//  * the warps quantise the piece's activations once into shared memory (31-bit
+//    block fixed point as two 16-bit digit planes, q4_intdot.cuh), then take
+//    units round-robin. Lane l owns block l of the unit's slice: its activation
+//    digits stay in registers while the slice does not change, and for each of
+//    the unit's rows it reads the block's 16 code bytes with one 128-bit shared
+//    load, forms sum_j (q_j - 8) X_j with 16 dp2a instructions, and applies the
+//    block's binary16 scale and power-of-two activation scale once. A slice
+//    holding a flagged block (an element the fixed point cannot carry within
+//    2^-14 of itself) is multiplied in binary32 instead;
 //  * the 8 rows of a unit are summed over the lanes with shuffles and written to
 //    per-(row, slice) shared slots; after the last unit each row's slices are
 //    added in slice order (deterministic) and y is stored, or, for a K split
@@ -34,6 +36,7 @@
 #include "q4_b1_plan.h"
 #include "q4_device.cuh"
 #include "q4_intdot.cuh"
+#include "q4_maps.h"
 
 using namespace q4dev;
 
@@ -42,55 +45,54 @@ namespace q4k {
 namespace {
 
 constexpr uint32_t kTimeoutFlag = 1u;
-constexpr int kConsumerBar = 1;  // named barrier of the consumer warps
+constexpr int kConsumerBar = 1;  // named barrier of the CTA's warps
 
 __device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "n"(q4b::kConsumers * 32) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "n"(q4b::kThreads) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-    uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return v;
-}
 
 __device__ __forceinline__ float half_bits_f32(uint32_t h) {
     return __half2float(__ushort_as_half((unsigned short)h));
 }
 
 // Quantise the piece's activations (all consumer threads): item i of
-// S * 32 * 8 is float4 g = i % 8 of block i / 8 (local slice (i / 8) / 32).
-// Eight consecutive lanes share a block; the block's largest |x|, digit sums and
-// flag are reduced over them with shuffles.
+// S * 32 * 8 is float4 g = i % 8 of block i / 8 (local slice (i / 8) / 32), and
+// thread `tid` takes items tid + 256 m, m < S. All of a thread's loads are issued
+// before any is used (one latency instead of S). Eight consecutive lanes share a
+// block; the block's largest |x|, digit sums and flag are reduced over them with
+// shuffles.
+constexpr int kMaxPieceSlices = 14;
+
 __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
-    const int items = S * q4b::kSliceBlocks * 8;
-    for (int base = 0; base < items; base += q4b::kConsumers * 32) {
-        const int i = base + tid;
+    float4 v[kMaxPieceSlices];
+#pragma unroll
+    for (int m = 0; m < kMaxPieceSlices; ++m) {
+        const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
         const int s = jl >> 5, jb = jl & 31;
-        const bool inside = i < items && jb < q4b::slice_blocks(G, s0 + s);
         const int64_t b = (int64_t)(s0 + s) * q4b::kSliceBlocks + jb;
-        const float4 v = inside ? __ldcg(reinterpret_cast<const float4*>(G.x + b * 32) + g)
-                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        uint32_t m = max(max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu),
-                         max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu));
+        v[m] = (m < S && jb < q4b::slice_blocks(G, s0 + s))
+                   ? __ldcg(reinterpret_cast<const float4*>(G.x + b * 32) + g)
+                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
 #pragma unroll
-        for (int off = 4; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int m = 0; m < kMaxPieceSlices; ++m) {
+        if (m >= S) break;
+        const int i = m * q4b::kWarps * 32 + tid;
+        const int jl = i >> 3, g = i & 7;
+        const int s = jl >> 5, jb = jl & 31;
+        uint32_t mx = max(max(__float_as_uint(v[m].x) & 0x7FFFFFFFu, __float_as_uint(v[m].y) & 0x7FFFFFFFu),
+                          max(__float_as_uint(v[m].z) & 0x7FFFFFFFu, __float_as_uint(v[m].w) & 0x7FFFFFFFu));
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         float sc, inv;
-        bool ok = xq_scale(m, &sc, &inv);
-        const float e[4] = {v.x, v.y, v.z, v.w};
+        bool ok = xq_scale(mx, &sc, &inv);
+        const float e[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
         int32_t d0[4], d1[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -107,16 +109,14 @@ __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8
             sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
             flag |= __shfl_xor_sync(0xffffffffu, flag, off);
         }
-        if (i < items) {
-            const uint32_t half = (uint32_t)(g & 1) * 8u;
-            *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, g >> 1, jb) + half) =
-                make_uint2(pack16(d0[0], d0[1]), pack16(d0[2], d0[3]));
-            *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, 4 + (g >> 1), jb) + half) =
-                make_uint2(pack16(d1[0], d1[1]), pack16(d1[2], d1[3]));
-            if (g == 0)
-                *reinterpret_cast<uint4*>(xs + q4b::xchunk_offset(s, 8, jb)) =
-                    make_uint4((uint32_t)(-8 * sum0), (uint32_t)(-8 * sum1), __float_as_uint(sc), flag);
-        }
+        const uint32_t half = (uint32_t)(g & 1) * 8u;
+        *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, g >> 1, jb) + half) =
+            make_uint2(pack16(d0[0], d0[1]), pack16(d0[2], d0[3]));
+        *reinterpret_cast<uint2*>(xs + q4b::xchunk_offset(s, 4 + (g >> 1), jb) + half) =
+            make_uint2(pack16(d1[0], d1[1]), pack16(d1[2], d1[3]));
+        if (g == 0)
+            *reinterpret_cast<uint4*>(xs + q4b::xchunk_offset(s, 8, jb)) =
+                make_uint4((uint32_t)(-8 * sum0), (uint32_t)(-8 * sum1), __float_as_uint(sc), flag);
     }
 }
 
@@ -145,7 +145,7 @@ __device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* ws,
                                              volatile int* abort_flag, int lane) {
-    if (mbar_wait_bounded(bar, parity)) return true;
+    if (mbar_wait_short_bounded(bar, parity)) return true;
     if (lane == 0) {
         atomicOr(ws, kTimeoutFlag);
         *abort_flag = 1;
@@ -153,33 +153,46 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uin
     return false;
 }
 
-// The producer warp: every unit of the piece, in order, into ring slot u % slots.
-__device__ __forceinline__ void produce(const q4b::Params& P, const q4b::Desc& G, const q4b::Piece& pc,
-                                        int s0, int S, uint8_t* ring, uint64_t* full, uint64_t* empty,
-                                        volatile int* abort_flag, int lane) {
-    const int T = q4b::piece_tiles(pc);
-    const int U = T * S;
-    const int slots = P.slots;
-    for (int u = 0; u < U; ++u) {
-        const int slot = u % slots, round = u / slots;
-        if (round > 0) {
-            const bool ok = wait_bounded(empty + slot, (uint32_t)(round - 1) & 1u, P.ws, abort_flag, lane);
-            if (!__all_sync(0xffffffffu, ok)) return;
-            // order the consumers' shared-memory reads of the slot before the copies
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        if (*abort_flag) return;
-        const int t = u / S, s = u - t * S;
-        const q4b::LaneCopy c = q4b::lane_copy(G, pc, t, s0 + s, lane);
-        const uint32_t bytes = c.active ? c.bytes : 0u;
-        const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
-        if (lane == 0) mbar_arrive_expect_tx(full + slot, total + P.tx_extra);
-        __syncwarp();
-        if (c.active)
-            bulk_g2s(ring + (size_t)slot * q4b::kSlotBytes + c.dst,
-                     (c.scales ? reinterpret_cast<const uint8_t*>(G.d) : G.qs) + c.src_off, c.bytes,
-                     full + slot);
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Issue the loads of unit u of a piece into ring slot u % slots (whole warp):
+// lane `lane_issue` loads the codes (and, with the scale map, the scales) as 2-D
+// boxes; without the scale map lanes 8..15 copy one row's scales each. Spreading
+// the issuing lane over units and warps keeps few copies in flight per thread.
+__device__ __forceinline__ void issue_unit(const q4b::Params& P, const q4b::Desc& G, const q4b::Piece& pc,
+                                           int s0, int S, int u, uint8_t* ring, uint64_t* full, int lane,
+                                           int lane_issue) {
+    const int slot = u % P.slots;
+    const int t = u / S, s = u - t * S;
+    const int gs = s0 + s;
+    const int32_t row0 = pc.r0 + t * q4b::kTileRows;
+    uint8_t* dst = ring + (size_t)slot * q4b::kSlotBytes;
+    uint32_t bytes = 0;
+    q4b::LaneCopy c;
+    c.active = false;
+    if (!G.d_map) {
+        c = q4b::lane_copy(G, pc, t, gs, lane);
+        c.active = c.active && c.scales;
+        bytes = c.active ? c.bytes : 0u;
     }
+    const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + q4b::kMapCodeBytes +
+                           (G.d_map ? q4b::kMapScaleBytes : 0u);
+    if (lane == lane_issue) {
+        mbar_arrive_expect_tx(full + slot, total + P.tx_extra);
+        tma_load_2d(dst, &P.qs_map[pc.g], gs * (q4b::kSliceBlocks * 4), row0, full + slot);
+        if (G.d_map)
+            tma_load_2d(dst + q4b::kSlotQs, &P.d_map[pc.g], gs * q4b::kSliceBlocks, row0, full + slot);
+    }
+    __syncwarp();
+    if (c.active)
+        bulk_g2s(dst + c.dst, reinterpret_cast<const uint8_t*>(G.d) + c.src_off, c.bytes, full + slot);
 }
 
 // Activation data of lane `lane` for local slice s.
@@ -190,11 +203,10 @@ struct LaneX {
 };
 
 __device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, LaneX* lx) {
-    const uint32_t base = smem_addr(xs);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint4 a = lds128(base + q4b::xchunk_offset(s, q, lane));
-        const uint4 b = lds128(base + q4b::xchunk_offset(s, 4 + q, lane));
+        const uint4 a = *reinterpret_cast<const uint4*>(xs + q4b::xchunk_offset(s, q, lane));
+        const uint4 b = *reinterpret_cast<const uint4*>(xs + q4b::xchunk_offset(s, 4 + q, lane));
         lx->p.a0[4 * q] = a.x;
         lx->p.a0[4 * q + 1] = a.y;
         lx->p.a0[4 * q + 2] = a.z;
@@ -204,7 +216,7 @@ __device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, 
         lx->p.a1[4 * q + 2] = b.z;
         lx->p.a1[4 * q + 3] = b.w;
     }
-    const uint4 k = lds128(base + q4b::xchunk_offset(s, 8, lane));
+    const uint4 k = *reinterpret_cast<const uint4*>(xs + q4b::xchunk_offset(s, 8, lane));
     lx->p.c0 = (int32_t)k.x;
     lx->p.c1 = (int32_t)k.y;
     lx->scale = __uint_as_float(k.z);
@@ -213,7 +225,7 @@ __device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, 
 
 }  // namespace
 
-__global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
+__global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const q4b::Piece pc = q4b::piece_of(P, blockIdx.x);
@@ -224,39 +236,36 @@ __global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Par
     const int U = T * S;
     const int slots = P.slots;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + q4b::kMaxSlots;
     float* red = reinterpret_cast<float*>(smem + q4b::red_offset());
     uint8_t* xs = smem + q4b::x_offset(P);
     uint8_t* ring = smem + q4b::ring_offset(P);
     __shared__ int abort_flag;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < slots; ++i) {
-            mbar_init(full + i, 1);
-            mbar_init(empty + i, 1);  // one consumer warp per use
-        }
+        for (int i = 0; i < slots; ++i) mbar_init(full + i, 1);
         abort_flag = 0;
         mbar_fence_init();
     }
     __syncthreads();
     pdl_launch_dependents();
 
-    if (warp == q4b::kConsumers) {
-        // weights never depend on an earlier kernel: stream before the wait
-        produce(P, G, pc, s0, S, ring, full, empty, &abort_flag, lane);
-        return;
-    }
+    // weights never depend on an earlier kernel: the first `slots` units are
+    // requested before the wait on the previous kernel (unit u by warp u % 8)
+    for (int u = warp; u < U && u < slots; u += q4b::kWarps)
+        issue_unit(P, G, pc, s0, S, u, ring, full, lane, (u >> 3) & 31);
 
     pdl_wait();
     const int tid = threadIdx.x;
     stage_x(G, s0, S, xs, tid);
     consumer_sync();
 
-    const uint32_t ring_base = smem_addr(ring);
+    volatile int* abort_v = &abort_flag;
     int cur = -1;
     LaneX lx;
-    volatile int* abort_v = &abort_flag;
-    for (int u = warp; u < U; u += q4b::kConsumers) {
+    // units of this warp requested so far: warp, warp + 8, ... < issued_end
+    int issued_end = min(U, slots);
+    int u = warp;
+    for (; u < U; u += q4b::kWarps) {
         if (*abort_v) break;
         const int t = u / S, s = u - t * S;
         if (s != cur) {
@@ -269,13 +278,13 @@ __global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Par
         const int gs = s0 + s;
         const int bs = q4b::slice_blocks(G, gs);
         const int nr = min(q4b::kTileRows, pc.r1 - pc.r0 - t * q4b::kTileRows);
-        const uint32_t sb = ring_base + (uint32_t)slot * q4b::kSlotBytes;
+        const uint8_t* sb = ring + (size_t)slot * q4b::kSlotBytes;
         float v[8];
         if (!lx.flagged) {
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                const uint4 q = lds128(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                const uint32_t dh = lds_u16(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
+                const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                const uint32_t dh = *reinterpret_cast<const uint16_t*>(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
                 const float dot = block_dot16(q, lx.p);
                 v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * lx.scale * dot : 0.0f;
             }
@@ -288,17 +297,29 @@ __global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Par
             const UnpackConsts k = unpack_consts_default();
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                const uint4 q = lds128(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                const uint32_t dh = lds_u16(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
+                const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                const uint32_t dh = *reinterpret_cast<const uint16_t*>(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
                 const float2 d2 = block_dot(q, xf, k);
                 v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
             }
         }
+        // the slot is read: refill it with unit u + slots (the proxy fence orders
+        // this warp's shared-memory reads before the copies' writes)
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty + slot);
+        if (u + slots < U) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue_unit(P, G, pc, s0, S, u + slots, ring, full, lane, ((u + slots) >> 3) & 31);
+            issued_end = u + slots + 1;
+        }
         const float row_sum = reduce8(v, lane);
         const int r = lane >> 2;
         if ((lane & 3) == 0 && r < nr) red[(t * q4b::kTileRows + r) * S + s] = row_sum;
+    }
+    if (*abort_v) {
+        // leave no copy in flight: wait (bounded) for the units this warp
+        // requested and did not read
+        for (; u < issued_end; u += q4b::kWarps)
+            mbar_wait_short_bounded(full + u % slots, (uint32_t)(u / slots) & 1u);
     }
     consumer_sync();
     if (*abort_v) return;
@@ -306,7 +327,7 @@ __global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Par
     // each row's slices in slice order
     const int rows = pc.r1 - pc.r0;
     if (G.splits == 1) {
-        for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+        for (int rl = tid; rl < rows; rl += q4b::kThreads) {
             float sum = 0.0f;
             for (int s = 0; s < S; ++s) sum += red[rl * S + s];
             G.y[pc.r0 + rl] = sum;
@@ -315,14 +336,14 @@ __global__ void __maxnreg__(112) gemv_b1_kernel(const __grid_constant__ q4b::Par
     }
     float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
     uint32_t* tickets = P.ws + G.ticket_off;
-    for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+    for (int rl = tid; rl < rows; rl += q4b::kThreads) {
         float sum = 0.0f;
         for (int s = 0; s < S; ++s) sum += red[rl * S + s];
         part[(int64_t)pc.split * G.n + pc.r0 + rl] = sum;
     }
     __threadfence();
     consumer_sync();
-    for (int rl = tid; rl < rows; rl += q4b::kConsumers * 32) {
+    for (int rl = tid; rl < rows; rl += q4b::kThreads) {
         const int64_t row = pc.r0 + rl;
         if (atomicAdd(tickets + row, 1u) == (uint32_t)G.splits - 1u) {
             __threadfence();
@@ -341,6 +362,23 @@ cudaError_t setup_b1_kernel(int optin_smem) {
     if (q4b::kSmemBudget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
     return cudaFuncSetAttribute(gemv_b1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 q4b::kSmemBudget);
+}
+
+// Tensor maps of one GEMV: the code plane as uint32 [n][k/8] in boxes of 128 x 8
+// (one unit: 8 rows x 512 bytes), and, when its row stride is a multiple of 16
+// bytes, the scale plane uint16 [n][k/32] in boxes of 32 x 8 (*d_map = 1).
+cudaError_t encode_b1_maps(CUtensorMap* qs_map, CUtensorMap* d_map, int32_t* d_ok, const uint8_t* qs,
+                           const uint16_t* d, int64_t n, int64_t k) {
+    cudaError_t e = encode_2d(qs_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, qs, (uint64_t)(k / 8), (uint64_t)n,
+                              (uint64_t)(k / 2), (uint32_t)(q4b::kSliceBlocks * 4), (uint32_t)q4b::kTileRows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    const int64_t nb = k / 32;
+    *d_ok = nb % 8 == 0 ? 1 : 0;
+    if (*d_ok)
+        e = encode_2d(d_map, CU_TENSOR_MAP_DATA_TYPE_UINT16, d, (uint64_t)nb, (uint64_t)n, (uint64_t)(nb * 2),
+                      (uint32_t)q4b::kSliceBlocks, (uint32_t)q4b::kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return e;
 }
 
 cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream) {

@@ -11,16 +11,21 @@
 // u = t * S + s is tile t, slice s of the piece's S slices (tile-major, so a
 // consumer warp that takes every 8th unit keeps one slice when S divides 8).
 //
-// Per CTA: one producer warp streams every unit's code bytes and binary16 scales
-// from HBM into a ring of shared-memory slots with bulk copies on the TMA
-// engine (one full and one empty mbarrier per slot); eight consumer warps take
-// units round-robin, multiply them with the piece's activations (quantised once
-// per piece into shared memory), and write per-(row, slice) partial sums to
-// shared memory; after the last unit the CTA adds each row's slices in slice
+// Per CTA: eight warps take units round-robin (unit u by warp u % 8). Every
+// unit's code bytes and binary16 scales come from HBM into ring slot u % slots
+// on the TMA engine, two 2-D tensor loads per unit (8 rows x 512 code bytes; 8
+// rows x 32 scales) completing on the slot's mbarrier (a scale plane whose row
+// stride is not a multiple of 16 bytes is copied row by row instead); the first
+// `slots` units are requested at kernel entry, and each warp, once it has read
+// unit u, requests unit u + slots into the slot it just freed. Warps multiply
+// units with the piece's activations (quantised once per piece into shared
+// memory) and write per-(row, slice) partial sums to shared memory; after the last unit the CTA adds each row's slices in slice
 // order and stores y (or a split-K partial, added up in split order by the last
 // split of the row to arrive). Two CTAs of consecutive launches fit one SM, so a
 // launch streams its weights in while the previous one finishes.
 #pragma once
+
+#include <cuda.h>
 
 #include <cstdint>
 
@@ -34,24 +39,30 @@
 
 namespace q4b {
 
-constexpr int kConsumers = 8;                 // consumer warps
-constexpr int kWarps = kConsumers + 1;        // + the producer warp
+constexpr int kWarps = 8;                     // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kTileRows = 8;                  // rows per unit
 constexpr int kSliceBlocks = 32;              // blocks per unit (one per lane)
 constexpr int kSlotQs = kTileRows * kSliceBlocks * 16;  // code bytes of a unit
 constexpr int kDRow = 80;                     // scale bytes per row in a slot (64 + alignment slack)
+constexpr int kDMapRow = 64;                  // scale bytes per row when loaded by the tensor map
 constexpr int kSlotBytes = kSlotQs + kTileRows * kDRow;
 constexpr int kXBlockBytes = 144;             // staged activation block: 32 digit words + 4 words
 constexpr int kXChunks = kXBlockBytes / 16;   // 16-byte chunks per staged block
 constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
+// Ring slots: a multiple of kWarps, so that every unit routed to a slot
+// (u = slot mod slots) belongs to the same warp, which both requests and waits
+// for it: the warp is never more than one phase ahead of the slot's barrier,
+// which a parity wait requires.
 constexpr int kMaxSlots = 24;
-constexpr int kMinSlots = 6;
-constexpr int kBarBytes = 2 * kMaxSlots * 8;  // full[], empty[]
+constexpr int kMinSlots = 8;
+constexpr int kBarBytes = 256;                // full[] barriers (kMaxSlots x 8 bytes), padded
 // Shared memory of one CTA: two CTAs of consecutive launches share an SM.
 constexpr int kSmemBudget = 113 * 1024;
 
 static_assert(kSlotBytes % 128 == 0, "slots keep 128-byte alignment");
+static_assert(kMaxSlots * 8 <= kBarBytes && kBarBytes % 128 == 0, "barrier region");
+static_assert(kMaxSlots % kWarps == 0 && kMinSlots % kWarps == 0, "slots per warp");
 static_assert(kXSliceBytes % 16 == 0, "staged slices keep 16-byte alignment");
 
 struct Desc {
@@ -66,6 +77,8 @@ struct Desc {
     int32_t slices_per_split;
     int32_t piece_begin;       // first piece (CTA) of this GEMV
     int32_t cps;               // pieces (CTAs) per split
+    int32_t d_map;             // 1: scales loaded by the tensor map (row stride % 16 == 0)
+    int32_t pad_;
     int64_t part_off;          // floats: split-K partial sums [splits][n]
     int64_t ticket_off;        // uint32: one ticket per row
 };
@@ -76,6 +89,10 @@ struct Piece {
 };
 
 struct Params {
+    // code plane as uint32 [n][k/8], box 128 x 8 rows; scale plane uint16
+    // [n][k/32], box 32 x 8 rows (used when Desc::d_map is set)
+    CUtensorMap qs_map[Q4_MAX_GROUP];
+    CUtensorMap d_map[Q4_MAX_GROUP];
     Desc g[Q4_MAX_GROUP];
     int32_t count;
     int32_t slots;             // ring slots of this launch
@@ -124,10 +141,16 @@ Q4B_HD int slice_blocks(const Desc& G, int gs) {
 
 Q4B_HD int piece_tiles(const Piece& p) { return (p.r1 - p.r0 + kTileRows - 1) / kTileRows; }
 
-// The copy lane `lane` of the producer issues for unit (tile t, local slice s)
-// of a piece: lanes 0..7 the code bytes of row r = lane, lanes 8..15 the
-// 16-byte aligned superset of that row's scales (the d plane is padded to 16
-// bytes, so a superset never leaves it).
+// Bytes one unit brings into its slot through the tensor maps: all 8 rows of the
+// box, rows and blocks past the ends read as zero.
+constexpr uint32_t kMapCodeBytes = kSlotQs;
+constexpr uint32_t kMapScaleBytes = kTileRows * kDMapRow;
+
+// The per-row copy lane `lane` of the producer issues for unit (tile t, global
+// slice gs) of a piece when the scales cannot use the tensor map: lanes 8..15 the
+// 16-byte aligned superset of row r = lane - 8's scales (the d plane is padded
+// to 16 bytes, so a superset never leaves it). Lanes 0..7 describe the code
+// bytes of row r = lane (loaded by the tensor map; the replay checks them).
 struct LaneCopy {
     int64_t src_off;  // byte offset in the qs plane (code copy) or the d plane
     uint32_t dst;     // byte offset inside a slot
@@ -159,6 +182,7 @@ Q4B_HD LaneCopy lane_copy(const Desc& G, const Piece& p, int t, int gs, int lane
 
 // Byte offset, inside a slot, of the scale of block `lane` of row r of the unit.
 Q4B_HD uint32_t scale_offset(const Desc& G, const Piece& p, int t, int gs, int r, int lane) {
+    if (G.d_map) return (uint32_t)(kSlotQs + r * kDMapRow + 2 * lane);
     const int64_t row = (int64_t)p.r0 + (int64_t)t * kTileRows + r;
     const int64_t a = (row * G.nb + (int64_t)gs * kSliceBlocks) * 2;
     return (uint32_t)(kSlotQs + r * kDRow + (int)(a & 15) + 2 * lane);

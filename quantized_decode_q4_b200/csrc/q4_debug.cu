@@ -53,7 +53,7 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
     if (plan_b1(sh, count, base, num_sms, &P, &tickets, &end) != Q4_OK) return 2;
     // shared memory: inside the budget, regions aligned, ring within its bounds
     if (smem_bytes(P) > (uint32_t)kSmemBudget) return 3;
-    if (P.slots < kMinSlots || P.slots > kMaxSlots) return 3;
+    if (P.slots < kMinSlots || P.slots > kMaxSlots || P.slots % kWarps) return 3;
     if (ring_offset(P) % 128 || x_offset(P) % 16 || red_offset() % 16) return 4;
     if (P.npieces < 1) return 5;
     {
@@ -91,23 +91,37 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
                 const int gs = s0 + s;
                 const int bs = slice_blocks(G, gs);
                 if (bs < 1 || bs > kSliceBlocks) return 12;
-                int64_t tx = 0;
-                for (int lane = 0; lane < 32; ++lane) {
-                    const LaneCopy lc = lane_copy(G, pc, t, gs, lane);
-                    const int r = lane & 7;
-                    const int64_t row = (int64_t)pc.r0 + (int64_t)t * kTileRows + r;
-                    if (lane >= 16 || row >= pc.r1) {
-                        if (lc.active) return 13;
-                        continue;
-                    }
-                    if (!lc.active) return 13;
-                    if (lc.src_off < 0 || lc.src_off % 16 || lc.bytes % 16 || lc.bytes == 0 || lc.dst % 16)
-                        return 14;
-                    if (!lc.scales) {
-                        if (lc.src_off + lc.bytes > qs_plane) return 15;
-                        if (lc.dst + lc.bytes > (uint32_t)((r + 1) * kSliceBlocks * 16)) return 16;
-                        if (lc.src_off != (row * G.nb + (int64_t)gs * kSliceBlocks) * 16) return 17;
-                    } else {
+                // codes: one box of 128 uint32 x 8 rows at (gs * 128, row0): its
+                // x coordinate is 16-byte aligned and it covers the unit's blocks
+                const int64_t row0 = (int64_t)pc.r0 + (int64_t)t * kTileRows;
+                if (((int64_t)gs * kSliceBlocks * 16) % 16 || row0 >= (int64_t(1) << 31)) return 14;
+                if ((int64_t)gs * kSliceBlocks * 16 >= sh[pc.g].k / 2) return 15;
+                if (kMapCodeBytes != (uint32_t)(kTileRows * kSliceBlocks * 16) || kMapCodeBytes > (uint32_t)kSlotQs)
+                    return 16;
+                int64_t tx = kMapCodeBytes;
+                if (G.d_map) {
+                    // scales: one box of 32 uint16 x 8 rows at (gs * 32, row0); the
+                    // plane's row stride must be a multiple of 16 bytes
+                    if ((G.nb * 2) % 16 || ((int64_t)gs * kSliceBlocks * 2) % 16) return 17;
+                    if (kMapScaleBytes > (uint32_t)(kTileRows * kDRow)) return 19;
+                    for (int r = 0; r < kTileRows; ++r)
+                        for (int j = 0; j < kSliceBlocks; ++j) {
+                            const uint32_t off = scale_offset(G, pc, t, gs, r, j);
+                            if (off != (uint32_t)(kSlotQs + (r * kSliceBlocks + j) * 2)) return 20;
+                        }
+                    tx += kMapScaleBytes;
+                } else {
+                    for (int lane = 8; lane < 16; ++lane) {
+                        const LaneCopy lc = lane_copy(G, pc, t, gs, lane);
+                        const int r = lane & 7;
+                        const int64_t row = row0 + r;
+                        if (row >= pc.r1) {
+                            if (lc.active) return 13;
+                            continue;
+                        }
+                        if (!lc.active || !lc.scales) return 13;
+                        if (lc.src_off < 0 || lc.src_off % 16 || lc.bytes % 16 || lc.bytes == 0 || lc.dst % 16)
+                            return 14;
                         if (lc.src_off + lc.bytes > d_plane) return 18;
                         if (lc.dst < (uint32_t)kSlotQs || lc.dst + lc.bytes > (uint32_t)(kSlotQs + (r + 1) * kDRow))
                             return 19;
@@ -118,9 +132,10 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
                             if (off < lc.dst || off + 2 > lc.dst + lc.bytes) return 20;
                             if ((int64_t)(off - lc.dst) + lc.src_off != want) return 20;
                         }
+                        tx += lc.bytes;
                     }
-                    tx += lc.bytes;
                 }
+                (void)qs_plane;
                 if (tx >= (int64_t(1) << 20)) return 21;
                 for (int r = 0; r < kTileRows; ++r) {
                     const int64_t row = (int64_t)pc.r0 + (int64_t)t * kTileRows + r;

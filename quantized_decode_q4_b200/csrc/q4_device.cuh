@@ -71,6 +71,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// The same bounded wait with try_wait at the hardware's own short time limit (no
+// suspend hint), so a waiting thread notices the phase change at once: for waits
+// on the critical path of a pipeline.
+__device__ __forceinline__ bool mbar_try_short(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_short_bounded(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_addr(bar);
+    if (mbar_try_short(addr, parity)) return true;
+    const uint64_t start = global_ns();
+    while (true) {
+        if (mbar_try_short(addr, parity)) return true;
+        if (global_ns() - start > kWaitLimitNs) return false;
+    }
+}
+
 // Global -> shared bulk copy through the TMA engine, completing on `bar`.
 // dst, src and bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,

@@ -18,6 +18,8 @@ cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int
                            int num_sms, cudaStream_t stream);
 cudaError_t setup_b1_kernel(int optin_smem);
 cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream);
+cudaError_t encode_b1_maps(CUtensorMap* qs_map, CUtensorMap* d_map, int32_t* d_ok, const uint8_t* qs,
+                           const uint16_t* d, int64_t n, int64_t k);
 cudaError_t setup_tc_kernels(int optin_smem);
 cudaError_t launch_tc(const q4t::Params& P, bool pdl, cudaStream_t stream);
 cudaError_t encode_tc_maps(q4t::Maps* maps, int32_t* d_box, const uint8_t* qs, const uint16_t* d,

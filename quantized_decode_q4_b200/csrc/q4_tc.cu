@@ -44,6 +44,7 @@
 #include <mutex>
 
 #include "q4_device.cuh"
+#include "q4_maps.h"
 #include "q4_tc_math.cuh"
 #include "q4_tc_plan.h"
 
@@ -146,7 +147,7 @@ struct Ctx {
 
 // Bounded wait of a single thread.
 __device__ __forceinline__ bool wait1(const Ctx& C, const q4t::Params& P, int b, uint32_t parity) {
-    if (mbar_wait_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity)) return true;
+    if (mbar_wait_short_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity)) return true;
     C.abort(P);
     return false;
 }
@@ -154,7 +155,7 @@ __device__ __forceinline__ bool wait1(const Ctx& C, const q4t::Params& P, int b,
 // Bounded wait of a whole warp; the outcome is the same for every lane.
 __device__ __forceinline__ bool waitw(const Ctx& C, const q4t::Params& P, int b, uint32_t parity) {
     const bool ok = __all_sync(0xffffffffu,
-                               mbar_wait_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity));
+                               mbar_wait_short_bounded(reinterpret_cast<uint64_t*>(C.smem + 8 * b), parity));
     if (!ok && (threadIdx.x & 31) == 0) C.abort(P);
     return ok;
 }
@@ -605,30 +606,6 @@ __global__ void __launch_bounds__(q4t::kThreads, 1) gemv_tc_kernel(const __grid_
 
 namespace {
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-std::mutex g_encode_mu;
-EncodeTiledFn g_encode = nullptr;
-
-EncodeTiledFn encode_fn() {
-    std::lock_guard<std::mutex> lock(g_encode_mu);
-    if (!g_encode) {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
-                cudaSuccess ||
-            qr != cudaDriverEntryPointSuccess)
-            return nullptr;
-        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-    return g_encode;
-}
-
 template <int BT>
 cudaError_t setup_one(int optin_smem) {
     cudaFuncAttributes fa;
@@ -659,23 +636,6 @@ cudaError_t launch_one(const q4t::Params& P, bool pdl, cudaStream_t stream) {
 // Token count a launch is compiled for: the smallest of 2, 4, 8, 16 >= b.
 int tc_tokens(int b) { return b <= 2 ? 2 : b <= 4 ? 4 : b <= 8 ? 8 : 16; }
 
-namespace {
-cudaError_t encode(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
-                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                   CUtensorMapSwizzle swizzle) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-}  // namespace
-
 // Tensor maps of one GEMV for b tokens (rows and columns past the ends read as
 // zero): code plane uint8 [n][k/2], box 128 B x 128 rows with the 128-byte
 // swizzle; activations binary32 [b][k], box 256 x (b rounded up to the compiled
@@ -683,18 +643,18 @@ cudaError_t encode(CUtensorMap* map, CUtensorMapDataType type, const void* base,
 // stride is a multiple of 16 bytes (*d_box = 1).
 cudaError_t encode_tc_maps(q4t::Maps* maps, int32_t* d_box, const uint8_t* qs, const uint16_t* d,
                            const float* x, int64_t n, int64_t k, int b) {
-    cudaError_t e = encode(&maps->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, qs, (uint64_t)(k / 2),
+    cudaError_t e = encode_2d(&maps->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, qs, (uint64_t)(k / 2),
                            (uint64_t)n, (uint64_t)(k / 2), 128u, (uint32_t)q4t::kM,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    e = encode(&maps->x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, (uint64_t)k, (uint64_t)b,
+    e = encode_2d(&maps->x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, (uint64_t)k, (uint64_t)b,
                (uint64_t)(k * 4), (uint32_t)(q4t::kS * 32), (uint32_t)tc_tokens(b),
                CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
     const int64_t nb = k / 32;
     *d_box = nb % 8 == 0 ? 1 : 0;
     if (*d_box)
-        e = encode(&maps->d, CU_TENSOR_MAP_DATA_TYPE_UINT16, d, (uint64_t)nb, (uint64_t)n,
+        e = encode_2d(&maps->d, CU_TENSOR_MAP_DATA_TYPE_UINT16, d, (uint64_t)nb, (uint64_t)n,
                    (uint64_t)(nb * 2), (uint32_t)q4t::kS, (uint32_t)q4t::kM,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
     return e;

@@ -69,7 +69,7 @@ def test_noalloc_rejects_matrices_beyond_its_scratch():
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     fn = _noalloc()
-    n, k = 64, 1 << 25   # split-K partial sums of about 2 MiB, beyond the 1 MiB array
+    n, k = 65536, 57344   # K in 4 splits: tickets and partial sums of 1.3 MB, beyond 1 MiB
     assert q4.workspace_bytes(n, k, 1) > (1 << 20)
     m = q4.q4_matrix(256, 256, n, k)  # never dereferenced: rejected before any launch
     assert fn(ctypes.byref(m), 256, 256, None) == 3
