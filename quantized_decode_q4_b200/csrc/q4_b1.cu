@@ -162,38 +162,55 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-// Issue the loads of unit u of a piece into ring slot u % slots (whole warp):
-// lane `lane_issue` loads the codes (and, with the scale map, the scales) as 2-D
-// boxes; without the scale map lanes 8..15 copy one row's scales each. Spreading
-// the issuing lane over units and warps keeps few copies in flight per thread.
+// Issue the loads of unit (tile t, local slice s) of a piece into ring slot
+// `slot` (whole warp): lane `lane_issue` loads the codes (and, with the scale
+// map, the scales) as 2-D boxes; without the scale map lanes 8..15 copy one row's
+// scales each. Spreading the issuing lane over units and warps keeps few copies
+// in flight per thread.
+template <bool kDMap>
 __device__ __forceinline__ void issue_unit(const q4b::Params& P, const q4b::Desc& G, const q4b::Piece& pc,
-                                           int s0, int S, int u, uint8_t* ring, uint64_t* full, int lane,
-                                           int lane_issue) {
-    const int slot = u % P.slots;
-    const int t = u / S, s = u - t * S;
-    const int gs = s0 + s;
+                                           int gsl, int t, int slot, uint8_t* ring, uint64_t* full,
+                                           int lane, int lane_issue) {
     const int32_t row0 = pc.r0 + t * q4b::kTileRows;
     uint8_t* dst = ring + (size_t)slot * q4b::kSlotBytes;
-    uint32_t bytes = 0;
-    q4b::LaneCopy c;
-    c.active = false;
-    if (!G.d_map) {
-        c = q4b::lane_copy(G, pc, t, gs, lane);
-        c.active = c.active && c.scales;
-        bytes = c.active ? c.bytes : 0u;
+    if (kDMap) {
+        if (lane == lane_issue) {
+            mbar_arrive_expect_tx(full + slot, q4b::kMapCodeBytes + q4b::kMapScaleBytes + P.tx_extra);
+            tma_load_2d(dst, &P.qs_map[pc.g], gsl * (q4b::kSliceBlocks * 4), row0, full + slot);
+            tma_load_2d(dst + q4b::kSlotQs, &P.d_map[pc.g], gsl * q4b::kSliceBlocks, row0, full + slot);
+        }
+        return;
     }
-    const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + q4b::kMapCodeBytes +
-                           (G.d_map ? q4b::kMapScaleBytes : 0u);
+    q4b::LaneCopy c = q4b::lane_copy(G, pc, t, gsl, lane);
+    c.active = c.active && c.scales;
+    const uint32_t bytes = c.active ? c.bytes : 0u;
+    const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + q4b::kMapCodeBytes;
     if (lane == lane_issue) {
         mbar_arrive_expect_tx(full + slot, total + P.tx_extra);
-        tma_load_2d(dst, &P.qs_map[pc.g], gs * (q4b::kSliceBlocks * 4), row0, full + slot);
-        if (G.d_map)
-            tma_load_2d(dst + q4b::kSlotQs, &P.d_map[pc.g], gs * q4b::kSliceBlocks, row0, full + slot);
+        tma_load_2d(dst, &P.qs_map[pc.g], gsl * (q4b::kSliceBlocks * 4), row0, full + slot);
     }
     __syncwarp();
     if (c.active)
         bulk_g2s(dst + c.dst, reinterpret_cast<const uint8_t*>(G.d) + c.src_off, c.bytes, full + slot);
 }
+
+// Position of a warp in its piece's unit sequence (unit u = t * S + s), moved
+// 8 units at a time without division.
+struct Cursor {
+    int t, s;
+    __device__ void set(int u, int S) {
+        t = u / S;
+        s = u - t * S;
+    }
+    __device__ void advance(int dt, int ds, int S) {
+        t += dt;
+        s += ds;
+        if (s >= S) {
+            s -= S;
+            ++t;
+        }
+    }
+};
 
 // Activation data of lane `lane` for local slice s.
 struct LaneX {
@@ -225,7 +242,8 @@ __device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, 
 
 }  // namespace
 
-__global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
+template <bool kDMap>
+__global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const q4b::Piece pc = q4b::piece_of(P, blockIdx.x);
@@ -235,6 +253,8 @@ __global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_
     const int T = q4b::piece_tiles(pc);
     const int U = T * S;
     const int slots = P.slots;
+    const int nb = G.nb;
+    const float* const xg_base = G.x;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     float* red = reinterpret_cast<float*>(smem + q4b::red_offset());
     uint8_t* xs = smem + q4b::x_offset(P);
@@ -249,10 +269,19 @@ __global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_
     __syncthreads();
     pdl_launch_dependents();
 
+    // the warp's units are u = warp + 8 k; cursors step 8 units at a time
+    const int dt8 = q4b::kWarps / S, ds8 = q4b::kWarps - dt8 * S;  // one step: kWarps units
     // weights never depend on an earlier kernel: the first `slots` units are
-    // requested before the wait on the previous kernel (unit u by warp u % 8)
-    for (int u = warp; u < U && u < slots; u += q4b::kWarps)
-        issue_unit(P, G, pc, s0, S, u, ring, full, lane, (u >> 3) & 31);
+    // requested before the wait on the previous kernel (unit u by warp u % 8,
+    // into slot u)
+    {
+        Cursor c;
+        c.set(warp, S);
+        for (int u = warp, k = 0; u < U && u < slots; u += q4b::kWarps, ++k) {
+            issue_unit<kDMap>(P, G, pc, s0 + c.s, c.t, u, ring, full, lane, k & 31);
+            c.advance(dt8, ds8, S);
+        }
+    }
 
     pdl_wait();
     const int tid = threadIdx.x;
@@ -262,44 +291,63 @@ __global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_
     volatile int* abort_v = &abort_flag;
     int cur = -1;
     LaneX lx;
-    // units of this warp requested so far: warp, warp + 8, ... < issued_end
+    // refills: unit u + slots goes to the slot unit u leaves (the same warp's)
+    Cursor cu, cr;
+    cu.set(warp, S);
+    cr.set(warp + slots, S);
+    int slot = warp;
+    uint32_t phase = 0;
     int issued_end = min(U, slots);
-    int u = warp;
-    for (; u < U; u += q4b::kWarps) {
+    int u = warp, k = 0;
+    for (; u < U; u += q4b::kWarps, ++k) {
         if (*abort_v) break;
-        const int t = u / S, s = u - t * S;
+        const int t = cu.t, s = cu.s;
         if (s != cur) {
             load_lane_x(xs, s, lane, &lx);
             cur = s;
         }
-        const int slot = u % slots;
-        const bool ok = wait_bounded(full + slot, (uint32_t)(u / slots) & 1u, P.ws, &abort_flag, lane);
+        const bool ok = wait_bounded(full + slot, phase, P.ws, &abort_flag, lane);
         if (!__all_sync(0xffffffffu, ok)) break;
         const int gs = s0 + s;
-        const int bs = q4b::slice_blocks(G, gs);
+        const int bs = min(q4b::kSliceBlocks, nb - gs * q4b::kSliceBlocks);
         const int nr = min(q4b::kTileRows, pc.r1 - pc.r0 - t * q4b::kTileRows);
         const uint8_t* sb = ring + (size_t)slot * q4b::kSlotBytes;
         float v[8];
         if (!lx.flagged) {
+            const float ls = lx.scale;
+            if (kDMap && bs == q4b::kSliceBlocks && nr == q4b::kTileRows) {
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                const uint32_t dh = *reinterpret_cast<const uint16_t*>(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
-                const float dot = block_dot16(q, lx.p);
-                v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * lx.scale * dot : 0.0f;
+                for (int r = 0; r < 8; ++r) {
+                    const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                    const uint32_t dh =
+                        *reinterpret_cast<const uint16_t*>(sb + q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane);
+                    v[r] = half_bits_f32(dh) * ls * block_dot16(q, lx.p);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                    const uint32_t dh = *reinterpret_cast<const uint16_t*>(
+                        sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
+                                    : q4b::scale_offset(G, pc, t, gs, r, lane)));
+                    const float dot = block_dot16(q, lx.p);
+                    v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * ls * dot : 0.0f;
+                }
             }
         } else {
             // exact path: binary32 products with the activations themselves
             float4 xf[8];
-            const float4* xg = reinterpret_cast<const float4*>(G.x + ((int64_t)gs * q4b::kSliceBlocks + lane) * 32);
+            const float4* xg = reinterpret_cast<const float4*>(xg_base + ((int64_t)gs * q4b::kSliceBlocks + lane) * 32);
 #pragma unroll
             for (int c = 0; c < 8; ++c) xf[c] = lane < bs ? __ldcg(xg + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const UnpackConsts k = unpack_consts_default();
+            const UnpackConsts kc = unpack_consts_default();
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                const uint32_t dh = *reinterpret_cast<const uint16_t*>(sb + q4b::scale_offset(G, pc, t, gs, r, lane));
-                const float2 d2 = block_dot(q, xf, k);
+                const uint32_t dh = *reinterpret_cast<const uint16_t*>(
+                    sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
+                                : q4b::scale_offset(G, pc, t, gs, r, lane)));
+                const float2 d2 = block_dot(q, xf, kc);
                 v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
             }
         }
@@ -308,18 +356,31 @@ __global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_
         __syncwarp();
         if (u + slots < U) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue_unit(P, G, pc, s0, S, u + slots, ring, full, lane, ((u + slots) >> 3) & 31);
+            issue_unit<kDMap>(P, G, pc, s0 + cr.s, cr.t, slot, ring, full, lane, (k + slots / q4b::kWarps) & 31);
             issued_end = u + slots + 1;
         }
         const float row_sum = reduce8(v, lane);
         const int r = lane >> 2;
         if ((lane & 3) == 0 && r < nr) red[(t * q4b::kTileRows + r) * S + s] = row_sum;
+        cu.advance(dt8, ds8, S);
+        cr.advance(dt8, ds8, S);
+        slot += q4b::kWarps;
+        if (slot >= slots) {
+            slot -= slots;
+            phase ^= 1u;
+        }
     }
     if (*abort_v) {
         // leave no copy in flight: wait (bounded) for the units this warp
         // requested and did not read
-        for (; u < issued_end; u += q4b::kWarps)
-            mbar_wait_short_bounded(full + u % slots, (uint32_t)(u / slots) & 1u);
+        for (; u < issued_end; u += q4b::kWarps) {
+            mbar_wait_short_bounded(full + slot, phase);
+            slot += q4b::kWarps;
+            if (slot >= slots) {
+                slot -= slots;
+                phase ^= 1u;
+            }
+        }
     }
     consumer_sync();
     if (*abort_v) return;
@@ -357,10 +418,12 @@ __global__ void __launch_bounds__(q4b::kThreads, 2) gemv_b1_kernel(const __grid_
 
 cudaError_t setup_b1_kernel(int optin_smem) {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_b1_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_b1_kernel<true>);
     if (e != cudaSuccess) return e;
     if (q4b::kSmemBudget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
-    return cudaFuncSetAttribute(gemv_b1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemv_b1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, q4b::kSmemBudget);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemv_b1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 q4b::kSmemBudget);
 }
 
@@ -392,7 +455,11 @@ cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_b1_kernel, P);
+    // the scale-map instantiation when every GEMV of the group has a scale map
+    bool all_maps = true;
+    for (int i = 0; i < P.count; ++i) all_maps = all_maps && P.g[i].d_map;
+    return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<true>, P)
+                    : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<false>, P);
 }
 
 }  // namespace q4k

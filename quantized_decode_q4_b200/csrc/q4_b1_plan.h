@@ -39,8 +39,15 @@
 
 namespace q4b {
 
-constexpr int kWarps = 8;                     // warps per CTA
+#ifndef Q4B_WARPS
+#define Q4B_WARPS 8  // warps per CTA
+#endif
+#ifndef Q4B_CTAS_PER_SM
+#define Q4B_CTAS_PER_SM 2  // CTAs of consecutive launches sharing an SM
+#endif
+constexpr int kWarps = Q4B_WARPS;
 constexpr int kThreads = kWarps * 32;
+constexpr int kCtasPerSm = Q4B_CTAS_PER_SM;
 constexpr int kTileRows = 8;                  // rows per unit
 constexpr int kSliceBlocks = 32;              // blocks per unit (one per lane)
 constexpr int kSlotQs = kTileRows * kSliceBlocks * 16;  // code bytes of a unit
@@ -54,11 +61,11 @@ constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
 // (u = slot mod slots) belongs to the same warp, which both requests and waits
 // for it: the warp is never more than one phase ahead of the slot's barrier,
 // which a parity wait requires.
-constexpr int kMaxSlots = 24;
-constexpr int kMinSlots = 8;
-constexpr int kBarBytes = 256;                // full[] barriers (kMaxSlots x 8 bytes), padded
+constexpr int kMaxSlots = 48 / kCtasPerSm / kWarps * kWarps;
+constexpr int kMinSlots = kWarps;
+constexpr int kBarBytes = (kMaxSlots * 8 + 127) / 128 * 128;  // full[] barriers, padded
 // Shared memory of one CTA: two CTAs of consecutive launches share an SM.
-constexpr int kSmemBudget = 113 * 1024;
+constexpr int kSmemBudget = (kCtasPerSm == 2 ? 113 : 226) * 1024;
 
 static_assert(kSlotBytes % 128 == 0, "slots keep 128-byte alignment");
 static_assert(kMaxSlots * 8 <= kBarBytes && kBarBytes % 128 == 0, "barrier region");
