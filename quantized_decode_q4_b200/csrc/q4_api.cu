@@ -33,6 +33,11 @@ constexpr int kMaxPieceSlices = 14;
 // Shared-memory bytes a piece's per-(row, slice) partial sums may take: more
 // rows per piece give it more pieces (CTAs).
 constexpr int64_t kRedPref = 8192;
+// Pieces (CTAs) of one launch per multiprocessor.
+#ifndef Q4B_PIECES_PER_SM
+#define Q4B_PIECES_PER_SM 2
+#endif
+constexpr int64_t kPiecesPerSm = Q4B_PIECES_PER_SM;
 }  // namespace
 
 bool cuda_failed(cudaError_t e) {
@@ -107,14 +112,15 @@ q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4
         wsplit[i] = std::min<int64_t>(nb, sps * q4b::kSliceBlocks);  // blocks of a split
     }
     if (kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
-    // spare CTAs (up to one per multiprocessor): to the GEMV whose pieces carry
-    // the most weight bytes, a split's worth of pieces at a time
+    // spare CTAs (up to kPiecesPerSm per multiprocessor): to the GEMV whose
+    // pieces carry the most weight bytes, a split's worth of pieces at a time
+    const int64_t target = (int64_t)num_sms * kPiecesPerSm;
     int64_t total = 0;
     for (int i = 0; i < count; ++i) total += P->g[i].splits * cps[i];
     while (true) {
         int best = -1;
         for (int i = 0; i < count; ++i) {
-            if (cps[i] >= sh[i].n || total + P->g[i].splits > num_sms) continue;
+            if (cps[i] >= sh[i].n || total + P->g[i].splits > target) continue;
             if (best < 0 || sh[i].n * wsplit[i] * cps[best] > sh[best].n * wsplit[best] * cps[i]) best = i;
         }
         if (best < 0) break;

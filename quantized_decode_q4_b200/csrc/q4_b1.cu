@@ -283,6 +283,13 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
         }
     }
 
+    // warm L2 with the piece's activations (a hint: they are read only after
+    // the wait, and L2 holds whatever the previous kernel wrote)
+    if (threadIdx.x == 32) {
+        const int64_t e0 = (int64_t)s0 * q4b::kSliceBlocks * 32;
+        const int64_t e1 = min((int64_t)(s0 + S) * q4b::kSliceBlocks * 32, (int64_t)nb * 32);
+        bulk_prefetch_l2(xg_base + e0, (uint32_t)((e1 - e0) * 4));
+    }
     pdl_wait();
     const int tid = threadIdx.x;
     stage_x(G, s0, S, xs, tid);

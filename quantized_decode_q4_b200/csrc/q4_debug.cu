@@ -66,7 +66,7 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
         }
         if (pb != P.npieces) return 5;
         for (int i = 0; i < count; ++i)
-            if (P.g[i].cps < P.g[i].n && P.npieces + P.g[i].splits <= num_sms) return 5;
+            if (P.g[i].cps < P.g[i].n && P.npieces + P.g[i].splits <= 2 * num_sms) return 5;
     }
     // coverage of every (row, global slice) and the copies of every unit
     std::vector<std::vector<uint8_t>> cover(count);

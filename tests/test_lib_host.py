@@ -131,8 +131,8 @@ def test_batch1_plans_replay_random_groups():
 
 def test_batch1_plan_properties():
     gate_up = q4.plan_info([(14336, 4096), (14336, 4096)])
-    # no K split, one piece per multiprocessor, no split-K scratch
-    assert gate_up["splits"] == [1, 1] and gate_up["pieces"] == 148
+    # no K split, two pieces per multiprocessor, no split-K scratch
+    assert gate_up["splits"] == [1, 1] and gate_up["pieces"] == 296
     assert gate_up["ws_bytes"] == 256
     assert gate_up["smem"] <= 113 * 1024          # two CTAs share an SM
     assert gate_up["slots"] >= 16                  # a deep weight ring
