@@ -51,10 +51,6 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "n"(q4b::kThreads) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 
 __device__ __forceinline__ float half_bits_f32(uint32_t h) {
     return __half2float(__ushort_as_half((unsigned short)h));
@@ -66,12 +62,10 @@ __device__ __forceinline__ float half_bits_f32(uint32_t h) {
 // before any is used (one latency instead of S). Eight consecutive lanes share a
 // block; the block's largest |x|, digit sums and flag are reduced over them with
 // shuffles.
-constexpr int kMaxPieceSlices = 14;
-
 __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
-    float4 v[kMaxPieceSlices];
+    float4 v[q4b::kMaxSlices];
 #pragma unroll
-    for (int m = 0; m < kMaxPieceSlices; ++m) {
+    for (int m = 0; m < q4b::kMaxSlices; ++m) {
         const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
         const int s = jl >> 5, jb = jl & 31;
@@ -81,7 +75,7 @@ __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8
                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 #pragma unroll
-    for (int m = 0; m < kMaxPieceSlices; ++m) {
+    for (int m = 0; m < q4b::kMaxSlices; ++m) {
         if (m >= S) break;
         const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
@@ -116,7 +110,7 @@ __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8
             make_uint2(pack16(d1[0], d1[1]), pack16(d1[2], d1[3]));
         if (g == 0)
             *reinterpret_cast<uint4*>(xs + q4b::xchunk_offset(s, 8, jb)) =
-                make_uint4((uint32_t)(-8 * sum0), (uint32_t)(-8 * sum1), __float_as_uint(sc), flag);
+                make_uint4((uint32_t)(-8 * sum0), (uint32_t)(-8 * sum1), __float_as_uint(sc * 0.0625f), flag);
     }
 }
 
@@ -402,8 +396,11 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
         }
         return;
     }
+    // K split: this piece's partial sums, then one ticket per row range (pieces
+    // j of every split cover the same rows); the CTA that arrives last adds the
+    // range's partials in split order and resets the ticket
     float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
-    uint32_t* tickets = P.ws + G.ticket_off;
+    uint32_t* ticket = P.ws + G.ticket_off + pc.j;
     for (int rl = tid; rl < rows; rl += q4b::kThreads) {
         float sum = 0.0f;
         for (int s = 0; s < S; ++s) sum += red[rl * S + s];
@@ -411,16 +408,18 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
     }
     __threadfence();
     consumer_sync();
+    __shared__ int last_split;
+    if (tid == 0) last_split = atomicAdd(ticket, 1u) == (uint32_t)G.splits - 1u;
+    consumer_sync();
+    if (!last_split) return;
+    __threadfence();
     for (int rl = tid; rl < rows; rl += q4b::kThreads) {
         const int64_t row = pc.r0 + rl;
-        if (atomicAdd(tickets + row, 1u) == (uint32_t)G.splits - 1u) {
-            __threadfence();
-            float sum = 0.0f;
-            for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
-            G.y[row] = sum;
-            tickets[row] = 0u;
-        }
+        float sum = 0.0f;
+        for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
+        G.y[row] = sum;
     }
+    if (tid == 0) *ticket = 0u;
 }
 
 cudaError_t setup_b1_kernel(int optin_smem) {

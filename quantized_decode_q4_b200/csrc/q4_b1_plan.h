@@ -4,10 +4,10 @@
 // A launch covers one dependency group (up to Q4_MAX_GROUP GEMVs). Its work is
 // cut into pieces, one per CTA: GEMV g owns pieces [piece_begin, piece_begin +
 // splits * cps), piece piece_begin + split * cps + j being rows
-// [n j / cps, n (j + 1) / cps) of K split `split` (K is split across CTAs for
-// narrow groups, whose rows are fewer than the CTAs of a launch, and for K beyond
-// 14 slices). Within a piece, K is walked in slices of 32
-// blocks (1024 weights, one block per lane) and rows in tiles of 8: unit
+// [n j / cps, n (j + 1) / cps) of K split `split`. K is split into ranges of a few
+// slices of 32 blocks (1024 weights, one block per lane; one slice per split by
+// default), so that the activations a piece stages stay small next to its
+// weights. Within a piece, K is walked in slices and rows in tiles of 8: unit
 // u = t * S + s is tile t, slice s of the piece's S slices (tile-major, so a
 // consumer warp that takes every 8th unit keeps one slice when S divides 8).
 //
@@ -20,8 +20,8 @@
 // unit u, requests unit u + slots into the slot it just freed. Warps multiply
 // units with the piece's activations (quantised once per piece into shared
 // memory) and write per-(row, slice) partial sums to shared memory; after the last unit the CTA adds each row's slices in slice
-// order and stores y (or a split-K partial, added up in split order by the last
-// split of the row to arrive). Two CTAs of consecutive launches fit one SM, so a
+// order and stores y (or a split-K partial; the last piece of a row range to
+// arrive adds the range's partials up in split order). Two CTAs of consecutive launches fit one SM, so a
 // launch streams its weights in while the previous one finishes.
 #pragma once
 
@@ -57,6 +57,9 @@ constexpr int kSlotBytes = kSlotQs + kTileRows * kDRow;
 constexpr int kXBlockBytes = 144;             // staged activation block: 32 digit words + 4 words
 constexpr int kXChunks = kXBlockBytes / 16;   // 16-byte chunks per staged block
 constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
+// Slices of one piece, at most (its activations are staged whole, and must leave
+// room for the weight ring).
+constexpr int kMaxSlices = 14;
 // Ring slots: a multiple of kWarps, so that every unit routed to a slot
 // (u = slot mod slots) belongs to the same warp, which both requests and waits
 // for it: the warp is never more than one phase ahead of the slot's barrier,
@@ -87,11 +90,12 @@ struct Desc {
     int32_t d_map;             // 1: scales loaded by the tensor map (row stride % 16 == 0)
     int32_t pad_;
     int64_t part_off;          // floats: split-K partial sums [splits][n]
-    int64_t ticket_off;        // uint32: one ticket per row
+    int64_t ticket_off;        // uint32: n words reserved; row range j (piece j of each split) uses word j
 };
 
 struct Piece {
     int32_t g, split;
+    int32_t j;                 // index within the split: pieces j of all splits share rows
     int32_t r0, r1;            // rows of GEMV g (< 2^31)
 };
 
@@ -121,6 +125,7 @@ Q4B_HD Piece piece_of(const PP& P, int c) {
     p.g = g;
     p.split = local / G.cps;
     const int j = local - p.split * G.cps;
+    p.j = j;
     p.r0 = (int32_t)(G.n * j / G.cps);
     p.r1 = (int32_t)(G.n * (j + 1) / G.cps);
     return p;

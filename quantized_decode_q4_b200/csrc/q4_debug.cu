@@ -77,6 +77,13 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
         const Desc& G = P.g[pc.g];
         if (pc.r0 < 0 || pc.r1 <= pc.r0 || pc.r1 > G.n) return 7;
         if (pc.split < 0 || pc.split >= G.splits) return 8;
+        // the ticket of the piece's row range: inside the GEMV's ticket words, and
+        // shared only with the pieces of the same rows in the other splits
+        if (pc.j < 0 || pc.j >= G.cps || pc.j >= G.n) return 8;
+        if (G.splits > 1) {
+            const Piece q0 = piece_of(P, G.piece_begin + pc.j);
+            if (q0.split != 0 || q0.j != pc.j || q0.r0 != pc.r0 || q0.r1 != pc.r1) return 8;
+        }
         int s0 = 0, S = 0;
         piece_slices(G, pc.split, &s0, &S);
         if (S < 1 || s0 + S > G.nslices) return 9;
@@ -251,7 +258,7 @@ int64_t q4_debug_check_intdot(uint64_t seed, int64_t blocks) {
         }
         double got;
         if (!flag) {
-            got = (double)block_dot16(q, xp) * (double)sc;
+            got = (double)block_dot16(q, xp) * (double)sc / 16.0;
             // per element 2^-14 of itself, plus the binary32 rounding of the block sum
             if (!(std::fabs(got - exact) <= abs_sum * (std::ldexp(1.0, -14) + std::ldexp(1.0, -23)) + 1e-300))
                 ++bad;

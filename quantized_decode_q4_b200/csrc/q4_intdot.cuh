@@ -20,8 +20,9 @@
 // 0..15 is exact in integers:
 //   sum_j (q_j - 8) X_j = 65536 S1 + S0,   Sp = sum_j q_j Dp_j - 8 sum_j Dp_j,
 // each sum_j q_j Dp_j a chain of dp2a instructions (two 16-bit digits times two
-// 8-bit codes per instruction). |S0| <= 2^23 and |S1| <= 2^22, so both convert
-// to binary32 exactly and one fused multiply-add forms the block sum.
+// 8-bit codes per instruction). |S0| <= 2^23 and |S1| <= 2^22, so 16 S0 and
+// 16 S1 (the form block_dot16 computes) convert to binary32 exactly and one
+// fused multiply-add forms 16 times the block sum.
 #pragma once
 
 #include <cstdint>
@@ -107,7 +108,7 @@ __host__ __device__ __forceinline__ uint32_t pack16(int32_t a, int32_t b) {
     return ((uint32_t)a & 0xFFFFu) | ((uint32_t)b << 16);
 }
 
-// Sum over the low (mode lo) or high (mode hi) two bytes of u (unsigned codes)
+// Sum over the low (mode lo) or high (mode hi) two bytes of u (unsigned bytes)
 // times the two signed 16-bit halves of a, plus acc.
 __host__ __device__ __forceinline__ int32_t dp2a_lo(uint32_t a, uint32_t u, int32_t acc) {
 #ifdef __CUDA_ARCH__
@@ -138,16 +139,20 @@ struct XPlanes {
     int32_t c0, c1;
 };
 
-// sum_j (q_j - 8) X_j of one block from its 16 code bytes, as 4 words (word w
+// 16 sum_j (q_j - 8) X_j of one block from its 16 code bytes, as 4 words (word w
 // holds bytes 4w..4w+3; byte m carries code 4w+m in its low nibble and code
-// 16+4w+m in its high nibble). Returned as binary32 (one rounding).
+// 16+4w+m in its high nibble). The high nibbles are multiplied in place (as
+// bytes 16 q, no shift), so the low-nibble sums are scaled by 16 before the two
+// are added: 16 Sp = 16 (sum_lo q Dp - 8 sum Dp) + sum_hi (16 q) Dp, with
+// |16 S0| <= 2^27 and |16 S1| <= 2^26 (exact in binary32). Returned as binary32
+// (one rounding).
 __host__ __device__ __forceinline__ float block_dot16(const uint4 q, const XPlanes& x) {
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
     int32_t s0 = x.c0, s1 = x.c1, h0 = 0, h1 = 0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-        const uint32_t lo = words[w] & 0x0F0F0F0Fu;         // codes 4w .. 4w+3
-        const uint32_t hi = (words[w] >> 4) & 0x0F0F0F0Fu;  // codes 16+4w .. 16+4w+3
+        const uint32_t lo = words[w] & 0x0F0F0F0Fu;  // codes 4w .. 4w+3
+        const uint32_t hi = words[w] & 0xF0F0F0F0u;  // 16 x codes 16+4w .. 16+4w+3
         s0 = dp2a_lo(x.a0[2 * w], lo, s0);
         s0 = dp2a_hi(x.a0[2 * w + 1], lo, s0);
         h0 = dp2a_lo(x.a0[8 + 2 * w], hi, h0);
@@ -157,7 +162,7 @@ __host__ __device__ __forceinline__ float block_dot16(const uint4 q, const XPlan
         h1 = dp2a_lo(x.a1[8 + 2 * w], hi, h1);
         h1 = dp2a_hi(x.a1[9 + 2 * w], hi, h1);
     }
-    return fmaf((float)(s1 + h1), 65536.0f, (float)(s0 + h0));
+    return fmaf((float)(s1 * 16 + h1), 65536.0f, (float)(s0 * 16 + h0));
 }
 
 // Quantise one block of 32 activations (host reference of the kernel's staging):
