@@ -34,8 +34,9 @@ def check_step(step: DecodeStep, rows_per_gemv: int, seed: int):
 
 @pytest.mark.parametrize("name,b", [("single_768", 1), ("minimind_26m", 1), ("minimind_26m", 2),
                                     ("minimind_26m", 8), ("minimind_26m", 16),
-                                    ("smollm2_135m", 1), ("gpt2_124m", 1),
-                                    ("smollm2_360m", 1), ("smollm2_360m", 4),
+                                    ("smollm2_135m", 1), ("smollm2_135m", 2),
+                                    ("smollm2_135m", 8), ("smollm2_135m", 16),
+                                    ("gpt2_124m", 1), ("smollm2_360m", 1), ("smollm2_360m", 4),
                                     ("smollm2_135m", 12)])
 def test_stack_parity(name, b):
     step = DecodeStep(synth.workloads()[name], b)
