@@ -28,9 +28,9 @@ extern "C" {
  * split-K tickets and partial sums must stay inside their workspace regions,
  * disjoint between GEMVs. Returns 0 when every check holds, otherwise the number
  * of the first failed check (see q4_debug.cu). */
-int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms);
+int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int num_sms);
 
-/* Summary of the batch-1 plan above for a 148-multiprocessor B200 (b must be 1):
+/* Summary of the CUDA-core plan above for a 148-multiprocessor B200 (1 <= b <= 4):
  * out[0] = CTAs (pieces), out[1] = dynamic shared memory bytes per CTA,
  * out[2] = workspace bytes, out[3] = weight ring slots, out[4 + i] = K splits of
  * GEMV i. Returns Q4_OK or Q4_ERR_INVALID_ARG. */

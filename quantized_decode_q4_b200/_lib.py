@@ -76,7 +76,7 @@ def lib():
             "q4_status_string": ([c.c_int], c.c_char_p),
             "q4_launch_count": ([], c.c_uint64),
             "q4_last_cuda_error": ([], c.c_char_p),
-            "q4_debug_check_b1": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int], c.c_int),
+            "q4_debug_check_b1": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int, c.c_int], c.c_int),
             "q4_gemv_noalloc": ([mp, vp, vp, vp], c.c_int),
             "q4_noalloc_status": ([vp], c.c_int),
             "q4_debug_plan_info": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int,
@@ -308,19 +308,20 @@ def status_string(s: int) -> str:
     return lib().q4_status_string(s).decode()
 
 
-def check_b1(shapes, num_sms: int = 148) -> int:
-    """Host replay of the batch-1 launch plan (0 when every check holds)."""
+def check_b1(shapes, num_sms: int = 148, b: int = 1) -> int:
+    """Host replay of the CUDA-core launch plan for b tokens (0 when every check
+    holds)."""
     n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
     k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
-    return lib().q4_debug_check_b1(n, k, len(shapes), num_sms)
+    return lib().q4_debug_check_b1(n, k, len(shapes), b, num_sms)
 
 
-def plan_info(shapes) -> dict:
-    """The batch-1 plan of one launch on a 148-SM B200."""
+def plan_info(shapes, b: int = 1) -> dict:
+    """The CUDA-core plan of one launch for b tokens on a 148-SM B200."""
     n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
     k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
     out = (ctypes.c_int64 * (4 + len(shapes)))()
-    _check(lib().q4_debug_plan_info(n, k, len(shapes), 1, out), "q4_debug_plan_info")
+    _check(lib().q4_debug_plan_info(n, k, len(shapes), b, out), "q4_debug_plan_info")
     return {"pieces": out[0], "smem": out[1], "ws_bytes": out[2], "slots": out[3],
             "splits": [out[4 + i] for i in range(len(shapes))]}
 

@@ -37,11 +37,6 @@ static_assert(kPieceSlices >= 1 && kPieceSlices <= q4b::kMaxSlices, "slices per 
 // Shared-memory bytes a piece's per-(row, slice) partial sums may take: more
 // rows per piece give it more pieces (CTAs).
 constexpr int64_t kRedPref = 8192;
-// Pieces (CTAs) of one launch per multiprocessor.
-#ifndef Q4B_PIECES_PER_SM
-#define Q4B_PIECES_PER_SM 2
-#endif
-constexpr int64_t kPiecesPerSm = Q4B_PIECES_PER_SM;
 }  // namespace
 
 bool cuda_failed(cudaError_t e) {
@@ -72,9 +67,10 @@ q4_status check_matrix(const q4_matrix* m) {
 // batch-1 plan
 // ---------------------------------------------------------------------------
 
-q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4b::Params* P,
+q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_sms, q4b::Params* P,
                   int64_t* tickets, int64_t* ws_end) {
-    if (count < 1 || count > Q4_MAX_GROUP || num_sms < 1) return Q4_ERR_INVALID_ARG;
+    if (count < 1 || count > Q4_MAX_GROUP || num_sms < 1 || b < 1 || b > q4b::kMaxTokens)
+        return Q4_ERR_INVALID_ARG;
     std::memset(P, 0, sizeof *P);
     int64_t R = 0;
     for (int i = 0; i < count; ++i) {
@@ -109,19 +105,19 @@ q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4
             G.ticket_off = kHeaderBytes / 4 + tick;
             tick += sh[i].n;
             G.part_off = part / 4;
-            part += round_up(splits * sh[i].n * 4, 256);
+            part += round_up(splits * b * sh[i].n * 4, 256);  // [splits][b][n]
         }
         max_slices = std::max<int>(max_slices, (int)sps);
-        // rows of one piece: its per-(row, slice) partial sums stay within kRedPref
+        // rows of one piece: its per-(token, row, slice) partial sums stay within kRedPref
         const int64_t max_rows = std::max<int64_t>(
-            q4b::kTileRows, kRedPref / 4 / sps / q4b::kTileRows * q4b::kTileRows);
+            q4b::kTileRows, kRedPref / 4 / sps / b / q4b::kTileRows * q4b::kTileRows);
         cps[i] = std::min<int64_t>(sh[i].n, ceil_div(sh[i].n, max_rows));
         wsplit[i] = std::min<int64_t>(nb, sps * q4b::kSliceBlocks);  // blocks of a split
     }
     if (kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
-    // spare CTAs (up to kPiecesPerSm per multiprocessor): to the GEMV whose
+    // spare CTAs (up to q4b::pieces_per_sm(b) per multiprocessor): to the GEMV whose
     // pieces carry the most weight bytes, a split's worth of pieces at a time
-    const int64_t target = (int64_t)num_sms * kPiecesPerSm;
+    const int64_t target = (int64_t)num_sms * q4b::pieces_per_sm(b);
     int64_t total = 0;
     for (int i = 0; i < count; ++i) total += P->g[i].splits * cps[i];
     while (true) {
@@ -143,15 +139,18 @@ q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4
         pb += G.splits * cps[i];
         const int64_t rows_max = ceil_div(sh[i].n, cps[i]);
         red_floats = std::max<int64_t>(red_floats,
-                                       ceil_div(rows_max, q4b::kTileRows) * q4b::kTileRows * G.slices_per_split);
+                                       ceil_div(rows_max, q4b::kTileRows) * q4b::kTileRows * G.slices_per_split * b);
     }
     P->count = count;
     P->npieces = (int32_t)total;
     P->red_bytes = (uint32_t)round_up(red_floats * 4, 128);
-    P->x_bytes = (uint32_t)(max_slices * q4b::kXSliceBytes);
-    const int64_t room = (int64_t)q4b::kSmemBudget - q4b::kBarBytes - P->red_bytes - P->x_bytes;
+    P->b = b;
+    P->max_slices = max_slices;
+    P->x_bytes = (uint32_t)(max_slices * (b == 1 ? q4b::kXSliceBytes : b * q4b::kXFSliceBytes));
+    const int64_t room = (int64_t)q4b::smem_budget(b) - q4b::kBarBytes - P->red_bytes - P->x_bytes;
     // a multiple of the CTA's warps: each slot is requested and read by one warp
-    const int64_t slots = std::min<int64_t>(room / q4b::kSlotBytes, q4b::kMaxSlots) / q4b::kWarps * q4b::kWarps;
+    const int64_t slots =
+        std::min<int64_t>(room / q4b::kSlotBytes, q4b::max_slots(b)) / q4b::kWarps * q4b::kWarps;
     if (slots < q4b::kMinSlots) return Q4_ERR_UNSUPPORTED;
     P->slots = (int32_t)slots;
     *tickets = tick;
@@ -219,9 +218,9 @@ q4_status group_need(const Shape* sh, int count, int b, int num_sms, int64_t* ti
     constexpr int64_t kBase = 0x40000000LL;
     int64_t t = 0, end = 0;
     q4_status s;
-    if (b == 1) {
+    if (b <= q4b::kMaxTokens) {
         q4b::Params P;
-        s = plan_b1(sh, count, kBase, num_sms, &P, &t, &end);
+        s = plan_b1(sh, count, b, kBase, num_sms, &P, &t, &end);
     } else {
         q4t::Params P;
         s = plan_tc(sh, count, b, kBase, num_sms, &P, &t, &end);
@@ -323,9 +322,9 @@ q4_status launch_group(const GemvCall* calls, int count, int b, void* ws, int64_
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {calls[i].m.n, calls[i].m.k};
     int64_t t = 0, end = 0;
-    if (b == 1) {
+    if (b <= q4b::kMaxTokens) {
         q4b::Params P;
-        q4_status s = plan_b1(sh, count, part_base, num_sms, &P, &t, &end);
+        q4_status s = plan_b1(sh, count, b, part_base, num_sms, &P, &t, &end);
         if (s != Q4_OK) return s;
         for (int i = 0; i < count; ++i) {
             P.g[i].qs = calls[i].m.qs;
@@ -436,9 +435,9 @@ q4_status gemv_call(const q4_matrix* m, const float* X, int b, float* Y, void* w
     if (s != Q4_OK) return s;
     if (!ws || ws_bytes < (size_t)kHeaderBytes) return Q4_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return Q4_ERR_MISALIGNED;
-    if (b == 1) {  // the batch-1 need does not depend on the device
+    if (b <= q4b::kMaxTokens) {  // the CUDA-core need does not depend on the device
         int64_t t = 0, p = 0;
-        if ((s = check_group(&call, 1, 1, 148, &t, &p)) != Q4_OK) return s;
+        if ((s = check_group(&call, 1, b, 148, &t, &p)) != Q4_OK) return s;
         if ((s = check_ws(ws, ws_bytes, (size_t)(part_base_for(t) + p))) != Q4_OK) return s;
     }
     int num_sms = 0;

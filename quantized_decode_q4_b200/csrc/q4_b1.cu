@@ -114,6 +114,40 @@ __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8
     }
 }
 
+// Copy the piece's activations of B tokens (2..4) into shared memory, binary32:
+// chunk c (values 4c .. 4c+3) of block j of local slice s of token t goes to
+// xfchunk_offset(s, t, B, c, j). Item i of a (slice, token) pair is chunk
+// 2 (w % 4) + (l % 2) of block 16 (w / 4) + l / 2 for i = 32 w + l, so two
+// neighbouring lanes read the two halves of one 32-byte sector; blocks past K are
+// staged as zeros. Loads go out eight rounds at a time before their stores.
+template <int B>
+__device__ __forceinline__ void stage_xf(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
+    static_assert(q4b::kThreads == 256, "one (slice, token) pair of 256 chunks per round");
+    const int64_t k = (int64_t)G.nb * 32;
+    const int rounds = S * B;  // one (slice, token) pair of 256 chunks per round
+    for (int m0 = 0; m0 < rounds; m0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int st = m0 + m, s = st / B, t = st - s * B;
+            const int w = tid >> 5, l = tid & 31;
+            const int c = ((w & 3) << 1) | (l & 1), jb = ((w >> 2) << 4) | (l >> 1);
+            v[m] = (st < rounds && jb < q4b::slice_blocks(G, s0 + s))
+                       ? __ldcg(reinterpret_cast<const float4*>(G.x + t * k +
+                                                                ((int64_t)(s0 + s) * q4b::kSliceBlocks + jb) * 32) + c)
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int st = m0 + m, s = st / B, t = st - s * B;
+            if (st >= rounds) break;
+            const int w = tid >> 5, l = tid & 31;
+            const int c = ((w & 3) << 1) | (l & 1), jb = ((w >> 2) << 4) | (l >> 1);
+            *reinterpret_cast<float4*>(xs + q4b::xfchunk_offset(s, t, B, c, jb)) = v[m];
+        }
+    }
+}
+
 // Sum each of 8 rows over the 32 lanes: afterwards lane l holds the total of
 // row l / 4 (lanes 4r .. 4r + 3 all hold row r).
 __device__ __forceinline__ float reduce8(float (&v)[8], int lane) {
@@ -236,8 +270,9 @@ __device__ __forceinline__ void load_lane_x(const uint8_t* xs, int s, int lane, 
 
 }  // namespace
 
-template <bool kDMap>
-__global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
+template <int B, bool kDMap>
+__global__ void __launch_bounds__(q4b::kThreads, q4b::ctas_per_sm(B))
+    gemv_b1_kernel(const __grid_constant__ q4b::Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const q4b::Piece pc = q4b::piece_of(P, blockIdx.x);
@@ -282,16 +317,23 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
     if (threadIdx.x == 32) {
         const int64_t e0 = (int64_t)s0 * q4b::kSliceBlocks * 32;
         const int64_t e1 = min((int64_t)(s0 + S) * q4b::kSliceBlocks * 32, (int64_t)nb * 32);
-        bulk_prefetch_l2(xg_base + e0, (uint32_t)((e1 - e0) * 4));
+#pragma unroll
+        for (int tk = 0; tk < B; ++tk)
+            bulk_prefetch_l2(xg_base + (int64_t)tk * nb * 32 + e0, (uint32_t)((e1 - e0) * 4));
     }
     pdl_wait();
     const int tid = threadIdx.x;
-    stage_x(G, s0, S, xs, tid);
+    if constexpr (B == 1)
+        stage_x(G, s0, S, xs, tid);
+    else
+        stage_xf<B>(G, s0, S, xs, tid);
     consumer_sync();
 
     volatile int* abort_v = &abort_flag;
     int cur = -1;
-    LaneX lx;
+    LaneX lx;                  // one token: digit planes
+    uint64_t xp[B][16];        // 2..4 tokens: binary32 pairs, chunk c as pairs 2c, 2c + 1
+    const UnpackConsts kc = unpack_consts_default();
     // refills: unit u + slots goes to the slot unit u leaves (the same warp's)
     Cursor cu, cr;
     cu.set(warp, S);
@@ -304,7 +346,19 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
         if (*abort_v) break;
         const int t = cu.t, s = cu.s;
         if (s != cur) {
-            load_lane_x(xs, s, lane, &lx);
+            if constexpr (B == 1) {
+                load_lane_x(xs, s, lane, &lx);
+            } else {
+#pragma unroll
+                for (int tk = 0; tk < B; ++tk)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 f =
+                            *reinterpret_cast<const float4*>(xs + q4b::xfchunk_offset(s, tk, B, c, lane));
+                        xp[tk][2 * c] = pack2(f.x, f.y);
+                        xp[tk][2 * c + 1] = pack2(f.z, f.w);
+                    }
+            }
             cur = s;
         }
         const bool ok = wait_bounded(full + slot, phase, P.ws, &abort_flag, lane);
@@ -313,8 +367,50 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
         const int bs = min(q4b::kSliceBlocks, nb - gs * q4b::kSliceBlocks);
         const int nr = min(q4b::kTileRows, pc.r1 - pc.r0 - t * q4b::kTileRows);
         const uint8_t* sb = ring + (size_t)slot * q4b::kSlotBytes;
-        float v[8];
-        if (!lx.flagged) {
+        float v[B][8];
+        if constexpr (B > 1) {
+            // each code word unpacked once into exact (q - 8) pairs, reused by
+            // every token with f32x2 fused multiply-adds
+            const bool whole = kDMap && bs == q4b::kSliceBlocks && nr == q4b::kTileRows;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
+                const uint32_t dh = *reinterpret_cast<const uint16_t*>(
+                    sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
+                                : q4b::scale_offset(G, pc, t, gs, r, lane)));
+                const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+                uint64_t acc[B][q4b::kTokenChains];
+#pragma unroll
+                for (int tk = 0; tk < B; ++tk)
+#pragma unroll
+                    for (int c = 0; c < q4b::kTokenChains; ++c) acc[tk][c] = 0ull;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint64_t pr[4];
+                    code_pairs(words[w], kc, pr);
+#pragma unroll
+                    for (int tk = 0; tk < B; ++tk) {
+                        uint64_t a = acc[tk][w % q4b::kTokenChains];
+                        a = ffma2(pr[0], xp[tk][2 * w], a);
+                        a = ffma2(pr[1], xp[tk][2 * w + 1], a);
+                        a = ffma2(pr[2], xp[tk][2 * w + 8], a);
+                        a = ffma2(pr[3], xp[tk][2 * w + 9], a);
+                        acc[tk][w % q4b::kTokenChains] = a;
+                    }
+                }
+                const float d = half_bits_f32(dh);
+                const bool live = whole || (lane < bs && r < nr);
+#pragma unroll
+                for (int tk = 0; tk < B; ++tk) {
+                    uint64_t a0 = acc[tk][0], a1 = acc[tk][1];
+                    if constexpr (q4b::kTokenChains == 4) {
+                        a0 = fadd2(a0, acc[tk][2]);
+                        a1 = fadd2(a1, acc[tk][3]);
+                    }
+                    v[tk][r] = live ? d * sum_pairs(a0, a1) : 0.0f;
+                }
+            }
+        } else if (!lx.flagged) {
             const float ls = lx.scale;
             if (kDMap && bs == q4b::kSliceBlocks && nr == q4b::kTileRows) {
 #pragma unroll
@@ -322,7 +418,7 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
                     const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
                     const uint32_t dh =
                         *reinterpret_cast<const uint16_t*>(sb + q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane);
-                    v[r] = half_bits_f32(dh) * ls * block_dot16(q, lx.p);
+                    v[0][r] = half_bits_f32(dh) * ls * block_dot16(q, lx.p);
                 }
             } else {
 #pragma unroll
@@ -332,7 +428,7 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
                         sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
                                     : q4b::scale_offset(G, pc, t, gs, r, lane)));
                     const float dot = block_dot16(q, lx.p);
-                    v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * ls * dot : 0.0f;
+                    v[0][r] = (lane < bs && r < nr) ? half_bits_f32(dh) * ls * dot : 0.0f;
                 }
             }
         } else {
@@ -341,7 +437,6 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
             const float4* xg = reinterpret_cast<const float4*>(xg_base + ((int64_t)gs * q4b::kSliceBlocks + lane) * 32);
 #pragma unroll
             for (int c = 0; c < 8; ++c) xf[c] = lane < bs ? __ldcg(xg + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const UnpackConsts kc = unpack_consts_default();
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
@@ -349,7 +444,7 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
                     sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
                                 : q4b::scale_offset(G, pc, t, gs, r, lane)));
                 const float2 d2 = block_dot(q, xf, kc);
-                v[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
+                v[0][r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
             }
         }
         // the slot is read: refill it with unit u + slots (the proxy fence orders
@@ -360,9 +455,12 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
             issue_unit<kDMap>(P, G, pc, s0 + cr.s, cr.t, slot, ring, full, lane, (k + slots / q4b::kWarps) & 31);
             issued_end = u + slots + 1;
         }
-        const float row_sum = reduce8(v, lane);
         const int r = lane >> 2;
-        if ((lane & 3) == 0 && r < nr) red[(t * q4b::kTileRows + r) * S + s] = row_sum;
+#pragma unroll
+        for (int tk = 0; tk < B; ++tk) {
+            const float row_sum = reduce8(v[tk], lane);
+            if ((lane & 3) == 0 && r < nr) red[((tk * T + t) * q4b::kTileRows + r) * S + s] = row_sum;
+        }
         cu.advance(dt8, ds8, S);
         cr.advance(dt8, ds8, S);
         slot += q4b::kWarps;
@@ -386,13 +484,15 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
     consumer_sync();
     if (*abort_v) return;
 
-    // each row's slices in slice order
+    // each (token, row)'s slices in slice order; y is [b][n]
     const int rows = pc.r1 - pc.r0;
+    const int T8 = T * q4b::kTileRows;
     if (G.splits == 1) {
-        for (int rl = tid; rl < rows; rl += q4b::kThreads) {
+        for (int i = tid; i < rows * B; i += q4b::kThreads) {
+            const int tk = i / rows, rl = i - tk * rows;
             float sum = 0.0f;
-            for (int s = 0; s < S; ++s) sum += red[rl * S + s];
-            G.y[pc.r0 + rl] = sum;
+            for (int s = 0; s < S; ++s) sum += red[(tk * T8 + rl) * S + s];
+            G.y[(int64_t)tk * G.n + pc.r0 + rl] = sum;
         }
         return;
     }
@@ -401,10 +501,11 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
     // range's partials in split order and resets the ticket
     float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
     uint32_t* ticket = P.ws + G.ticket_off + pc.j;
-    for (int rl = tid; rl < rows; rl += q4b::kThreads) {
+    for (int i = tid; i < rows * B; i += q4b::kThreads) {
+        const int tk = i / rows, rl = i - tk * rows;
         float sum = 0.0f;
-        for (int s = 0; s < S; ++s) sum += red[rl * S + s];
-        part[(int64_t)pc.split * G.n + pc.r0 + rl] = sum;
+        for (int s = 0; s < S; ++s) sum += red[(tk * T8 + rl) * S + s];
+        part[((int64_t)pc.split * B + tk) * G.n + pc.r0 + rl] = sum;
     }
     __threadfence();
     consumer_sync();
@@ -413,24 +514,36 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::kCtasPerSm) gemv_b1_kernel
     consumer_sync();
     if (!last_split) return;
     __threadfence();
-    for (int rl = tid; rl < rows; rl += q4b::kThreads) {
-        const int64_t row = pc.r0 + rl;
+    for (int i = tid; i < rows * B; i += q4b::kThreads) {
+        const int tk = i / rows;
+        const int64_t row = pc.r0 + (i - tk * rows);
         float sum = 0.0f;
-        for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
-        G.y[row] = sum;
+        for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + ((int64_t)sp * B + tk) * G.n + row);
+        G.y[(int64_t)tk * G.n + row] = sum;
     }
     if (tid == 0) *ticket = 0u;
 }
 
-cudaError_t setup_b1_kernel(int optin_smem) {
+namespace {
+template <int B>
+cudaError_t setup_b1_tokens(int optin_smem) {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_b1_kernel<true>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemv_b1_kernel<B, true>);
     if (e != cudaSuccess) return e;
-    if (q4b::kSmemBudget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(gemv_b1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, q4b::kSmemBudget);
+    const int budget = q4b::smem_budget(B);
+    if (budget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(gemv_b1_kernel<B, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, budget);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(gemv_b1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                q4b::kSmemBudget);
+    return cudaFuncSetAttribute(gemv_b1_kernel<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, budget);
+}
+}  // namespace
+
+cudaError_t setup_b1_kernel(int optin_smem) {
+    cudaError_t e = setup_b1_tokens<1>(optin_smem);
+    if (e == cudaSuccess) e = setup_b1_tokens<2>(optin_smem);
+    if (e == cudaSuccess) e = setup_b1_tokens<3>(optin_smem);
+    if (e == cudaSuccess) e = setup_b1_tokens<4>(optin_smem);
+    return e;
 }
 
 // Tensor maps of one GEMV: the code plane as uint32 [n][k/8] in boxes of 128 x 8
@@ -464,8 +577,22 @@ cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream) {
     // the scale-map instantiation when every GEMV of the group has a scale map
     bool all_maps = true;
     for (int i = 0; i < P.count; ++i) all_maps = all_maps && P.g[i].d_map;
-    return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<true>, P)
-                    : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<false>, P);
+    switch (P.b) {
+        case 1:
+            return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<1, true>, P)
+                            : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<1, false>, P);
+        case 2:
+            return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<2, true>, P)
+                            : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<2, false>, P);
+        case 3:
+            return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<3, true>, P)
+                            : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<3, false>, P);
+        case 4:
+            return all_maps ? cudaLaunchKernelEx(&cfg, gemv_b1_kernel<4, true>, P)
+                            : cudaLaunchKernelEx(&cfg, gemv_b1_kernel<4, false>, P);
+        default:
+            return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace q4k

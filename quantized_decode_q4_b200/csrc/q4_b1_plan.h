@@ -33,8 +33,10 @@
 
 #if defined(__CUDACC__)
 #define Q4B_HD __host__ __device__ __forceinline__
+#define Q4B_HD_CONST __host__ __device__ constexpr
 #else
 #define Q4B_HD inline
+#define Q4B_HD_CONST constexpr
 #endif
 
 namespace q4b {
@@ -43,20 +45,38 @@ namespace q4b {
 #define Q4B_WARPS 8  // warps per CTA
 #endif
 #ifndef Q4B_CTAS_PER_SM
-#define Q4B_CTAS_PER_SM 2  // CTAs of consecutive launches sharing an SM
+#define Q4B_CTAS_PER_SM 2  // CTAs of consecutive launches sharing an SM (1 and 2 tokens)
 #endif
 constexpr int kWarps = Q4B_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCtasPerSm = Q4B_CTAS_PER_SM;
+// Tokens one launch of this kernel multiplies, at most (one pass over the weights).
+#ifndef Q4B_MAX_TOKENS
+#define Q4B_MAX_TOKENS 4
+#endif
+constexpr int kMaxTokens = Q4B_MAX_TOKENS;
+#ifndef Q4B_CTAS_PER_SM_B2
+#define Q4B_CTAS_PER_SM_B2 Q4B_CTAS_PER_SM
+#endif
+// Accumulator chains per token and row of the 2..4-token path (2 or 4).
+#ifndef Q4B_TOKEN_CHAINS
+#define Q4B_TOKEN_CHAINS 2
+#endif
+constexpr int kTokenChains = Q4B_TOKEN_CHAINS;
+static_assert(kTokenChains == 2 || kTokenChains == 4, "accumulator chains");
+// CTAs per SM for b tokens: three and four tokens keep 32 b activation values per
+// lane in registers, which takes the register file of a whole SM.
+Q4B_HD_CONST int ctas_per_sm(int b) { return b == 1 ? kCtasPerSm : (b == 2 ? Q4B_CTAS_PER_SM_B2 : 1); }
 constexpr int kTileRows = 8;                  // rows per unit
 constexpr int kSliceBlocks = 32;              // blocks per unit (one per lane)
 constexpr int kSlotQs = kTileRows * kSliceBlocks * 16;  // code bytes of a unit
 constexpr int kDRow = 80;                     // scale bytes per row in a slot (64 + alignment slack)
 constexpr int kDMapRow = 64;                  // scale bytes per row when loaded by the tensor map
 constexpr int kSlotBytes = kSlotQs + kTileRows * kDRow;
-constexpr int kXBlockBytes = 144;             // staged activation block: 32 digit words + 4 words
+constexpr int kXBlockBytes = 144;             // staged activation block (1 token): 32 digit words + 4 words
 constexpr int kXChunks = kXBlockBytes / 16;   // 16-byte chunks per staged block
 constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
+constexpr int kXFSliceBytes = kSliceBlocks * 128;  // one token's slice in binary32 (2..4 tokens)
 // Slices of one piece, at most (its activations are staged whole, and must leave
 // room for the weight ring).
 constexpr int kMaxSlices = 14;
@@ -64,16 +84,23 @@ constexpr int kMaxSlices = 14;
 // (u = slot mod slots) belongs to the same warp, which both requests and waits
 // for it: the warp is never more than one phase ahead of the slot's barrier,
 // which a parity wait requires.
-constexpr int kMaxSlots = 48 / kCtasPerSm / kWarps * kWarps;
+// Pieces (CTAs) of one launch per multiprocessor: as many as fit at once.
+#ifndef Q4B_PIECES_PER_SM
+#define Q4B_PIECES_PER_SM 2
+#endif
+Q4B_HD_CONST int pieces_per_sm(int b) { return ctas_per_sm(b) == 2 ? Q4B_PIECES_PER_SM : 1; }
+Q4B_HD_CONST int max_slots(int b) { return 48 / ctas_per_sm(b) / kWarps * kWarps; }
+constexpr int kMaxSlots = 48 / kWarps * kWarps;  // over every token count
 constexpr int kMinSlots = kWarps;
 constexpr int kBarBytes = (kMaxSlots * 8 + 127) / 128 * 128;  // full[] barriers, padded
 // Shared memory of one CTA: two CTAs of consecutive launches share an SM.
-constexpr int kSmemBudget = (kCtasPerSm == 2 ? 113 : 226) * 1024;
+Q4B_HD_CONST int smem_budget(int b) { return (ctas_per_sm(b) == 2 ? 113 : 226) * 1024; }
 
 static_assert(kSlotBytes % 128 == 0, "slots keep 128-byte alignment");
 static_assert(kMaxSlots * 8 <= kBarBytes && kBarBytes % 128 == 0, "barrier region");
 static_assert(kMaxSlots % kWarps == 0 && kMinSlots % kWarps == 0, "slots per warp");
 static_assert(kXSliceBytes % 16 == 0, "staged slices keep 16-byte alignment");
+static_assert(kCtasPerSm == 1 || kCtasPerSm == 2, "one or two CTAs per SM");
 
 struct Desc {
     const uint8_t* qs;
@@ -111,6 +138,8 @@ struct Params {
     uint32_t x_bytes;          // shared memory for the staged activations
     uint32_t tx_extra;         // 0; test hook: bytes every slot waits for beyond its copies
     int32_t npieces;
+    int32_t b;                 // tokens (1 .. kMaxTokens); x [b][k], y [b][n]
+    int32_t max_slices;        // slices of the largest piece (staging stride of a token)
     uint32_t* ws;
 };
 
@@ -198,6 +227,13 @@ Q4B_HD uint32_t scale_offset(const Desc& G, const Piece& p, int t, int gs, int r
     const int64_t row = (int64_t)p.r0 + (int64_t)t * kTileRows + r;
     const int64_t a = (row * G.nb + (int64_t)gs * kSliceBlocks) * 2;
     return (uint32_t)(kSlotQs + r * kDRow + (int)(a & 15) + 2 * lane);
+}
+
+// Staged activations of tokens 2..4: chunk c (values 4c .. 4c+3) of block j of
+// local slice s of token t, binary32, at x_offset + (((s * b + t) * 8 + c) * 32 +
+// j) * 16 (the 32 lanes of a warp read 32 consecutive chunks).
+Q4B_HD uint32_t xfchunk_offset(int s, int t, int b, int c, int j) {
+    return (uint32_t)((((s * b + t) * 8 + c) * kSliceBlocks + j) * 16);
 }
 
 // Staged activation block j of local slice s: chunk q (0..8) of 16 bytes at

@@ -41,19 +41,20 @@ uint64_t splitmix(uint64_t* z) {
 
 extern "C" {
 
-int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms) {
+int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int num_sms) {
     using namespace q4b;
-    if (!n || !k || count < 1 || count > Q4_MAX_GROUP || num_sms < 1) return 1;
+    if (!n || !k || count < 1 || count > Q4_MAX_GROUP || num_sms < 1 || b < 1 || b > kMaxTokens) return 1;
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
     Params P;
     int64_t tickets = 0, end = 0;
-    if (plan_b1(sh, count, INT64_MAX / 4, num_sms, &P, &tickets, &end) != Q4_OK) return 2;
+    if (plan_b1(sh, count, b, INT64_MAX / 4, num_sms, &P, &tickets, &end) != Q4_OK) return 2;
     const int64_t base = part_base_for(tickets);
-    if (plan_b1(sh, count, base, num_sms, &P, &tickets, &end) != Q4_OK) return 2;
+    if (plan_b1(sh, count, b, base, num_sms, &P, &tickets, &end) != Q4_OK) return 2;
+    if (P.b != b) return 2;
     // shared memory: inside the budget, regions aligned, ring within its bounds
-    if (smem_bytes(P) > (uint32_t)kSmemBudget) return 3;
-    if (P.slots < kMinSlots || P.slots > kMaxSlots || P.slots % kWarps) return 3;
+    if (smem_bytes(P) > (uint32_t)smem_budget(b)) return 3;
+    if (P.slots < kMinSlots || P.slots > max_slots(b) || P.slots % kWarps) return 3;
     if (ring_offset(P) % 128 || x_offset(P) % 16 || red_offset() % 16) return 4;
     if (P.npieces < 1) return 5;
     {
@@ -66,7 +67,7 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
         }
         if (pb != P.npieces) return 5;
         for (int i = 0; i < count; ++i)
-            if (P.g[i].cps < P.g[i].n && P.npieces + P.g[i].splits <= 2 * num_sms) return 5;
+            if (P.g[i].cps < P.g[i].n && P.npieces + P.g[i].splits <= pieces_per_sm(b) * num_sms) return 5;
     }
     // coverage of every (row, global slice) and the copies of every unit
     std::vector<std::vector<uint8_t>> cover(count);
@@ -87,10 +88,17 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
         int s0 = 0, S = 0;
         piece_slices(G, pc.split, &s0, &S);
         if (S < 1 || s0 + S > G.nslices) return 9;
-        if ((uint32_t)S * kXSliceBytes > P.x_bytes) return 10;
-        if (xchunk_offset(S - 1, kXChunks - 1, kSliceBlocks - 1) + 16 > P.x_bytes) return 10;
+        if (b == 1) {
+            if ((uint32_t)S * kXSliceBytes > P.x_bytes) return 10;
+            if (xchunk_offset(S - 1, kXChunks - 1, kSliceBlocks - 1) + 16 > P.x_bytes) return 10;
+        } else {
+            if ((uint32_t)(S * b * kXFSliceBytes) > P.x_bytes) return 10;
+            if (xfchunk_offset(S - 1, b - 1, b, 7, kSliceBlocks - 1) + 16 > P.x_bytes) return 10;
+            // the staging rounds: one (slice, token) pair per 256 threads
+            if (kThreads != 256) return 10;
+        }
         const int T = piece_tiles(pc);
-        if ((int64_t)T * kTileRows * S * 4 > (int64_t)P.red_bytes) return 11;
+        if ((int64_t)T * kTileRows * S * b * 4 > (int64_t)P.red_bytes) return 11;
         const int64_t qs_plane = sh[pc.g].n * (sh[pc.g].k / 2);
         const int64_t d_plane = round_up(sh[pc.g].n * G.nb * 2, 16);
         for (int t = 0; t < T; ++t)
@@ -162,12 +170,13 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
         if (G.splits < 1 || (int64_t)G.splits * G.slices_per_split < G.nslices) return 24;
         if (G.splits == 1) continue;
         if (G.ticket_off * 4 < kHeaderBytes || (G.ticket_off + G.n) * 4 > base) return 25;
-        if (G.part_off * 4 < base || (G.part_off + (int64_t)G.splits * G.n) * 4 > end) return 26;
+        if (G.part_off * 4 < base || (G.part_off + (int64_t)G.splits * b * G.n) * 4 > end) return 26;
         for (int j = i + 1; j < count; ++j) {
             const Desc& H = P.g[j];
             if (H.splits == 1) continue;
             if (G.ticket_off < H.ticket_off + H.n && H.ticket_off < G.ticket_off + G.n) return 27;
-            if (G.part_off < H.part_off + H.splits * H.n && H.part_off < G.part_off + G.splits * G.n)
+            if (G.part_off < H.part_off + (int64_t)H.splits * b * H.n &&
+                H.part_off < G.part_off + (int64_t)G.splits * b * G.n)
                 return 27;
         }
     }
@@ -175,15 +184,16 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int num_sms
 }
 
 q4_status q4_debug_plan_info(const int64_t* n, const int64_t* k, int count, int b, int64_t* out) {
-    if (!n || !k || !out || count < 1 || count > Q4_MAX_GROUP || b != 1) return Q4_ERR_INVALID_ARG;
+    if (!n || !k || !out || count < 1 || count > Q4_MAX_GROUP || b < 1 || b > q4b::kMaxTokens)
+        return Q4_ERR_INVALID_ARG;
     Shape sh[Q4_MAX_GROUP];
     for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
     q4b::Params P;
     int64_t tickets = 0, end = 0;
-    q4_status s = plan_b1(sh, count, INT64_MAX / 4, kRefSms, &P, &tickets, &end);
+    q4_status s = plan_b1(sh, count, b, INT64_MAX / 4, kRefSms, &P, &tickets, &end);
     if (s != Q4_OK) return s;
     const int64_t base = part_base_for(tickets);
-    if ((s = plan_b1(sh, count, base, kRefSms, &P, &tickets, &end)) != Q4_OK) return s;
+    if ((s = plan_b1(sh, count, b, base, kRefSms, &P, &tickets, &end)) != Q4_OK) return s;
     out[0] = P.npieces;
     out[1] = q4b::smem_bytes(P);
     out[2] = end;

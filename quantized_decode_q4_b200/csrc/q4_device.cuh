@@ -273,4 +273,55 @@ __host__ __device__ __forceinline__ float2 block_dot(const uint4 q, const float4
     return acc;
 }
 
+#if defined(__CUDACC__)
+// The four exact binary32 pairs (q - 8) of one code word, in the order block_dot
+// uses them: (codes 4w, 4w+1), (4w+2, 4w+3), (16+4w, 16+4w+1), (16+4w+2,
+// 16+4w+3) for word w of a block, each pair as the two halves of a 64-bit
+// register (low half first). Several token rows reuse them.
+__device__ __forceinline__ void code_pairs(uint32_t word, const UnpackConsts& k, uint64_t (&p)[4]) {
+    asm("{\n"
+        " .reg .b32 s, t0, t1;\n"
+        " shr.b32 s, %4, 12;\n"
+        " lop3.b32 t0, %4, 0x0000000F, %5, 0xEA;\n"
+        " lop3.b32 t1, %4, 0x00000F00, %7, 0xEA;\n"
+        " mov.b64 %0, {t0, t1};\n add.rn.f32x2 %0, %0, %10;\n"
+        " lop3.b32 t0, %4, 0x000F0000, %9, 0xEA;\n"
+        " lop3.b32 t1, s, 0x0000F000, %8, 0xEA;\n"
+        " mov.b64 %1, {t0, t1};\n add.rn.f32x2 %1, %1, %11;\n"
+        " lop3.b32 t0, %4, 0x000000F0, %6, 0xEA;\n"
+        " lop3.b32 t1, %4, 0x0000F000, %8, 0xEA;\n"
+        " mov.b64 %2, {t0, t1};\n add.rn.f32x2 %2, %2, %12;\n"
+        " lop3.b32 t0, s, 0x00000F00, %7, 0xEA;\n"
+        " lop3.b32 t1, s, 0x000F0000, %9, 0xEA;\n"
+        " mov.b64 %3, {t0, t1};\n add.rn.f32x2 %3, %3, %13;\n"
+        "}\n"
+        : "=l"(p[0]), "=l"(p[1]), "=l"(p[2]), "=l"(p[3])
+        : "r"(word), "r"(k.e23), "r"(k.e19), "r"(k.e15), "r"(k.e11), "r"(k.e7), "l"(k.lo01), "l"(k.lo23),
+          "l"(k.hi01), "l"(k.hi23));
+}
+
+// c + a * b on both halves of 64-bit registers holding binary32 pairs.
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+
+// Sum of the four binary32 values in two pairs: (a.lo + b.lo) + (a.hi + b.hi).
+__device__ __forceinline__ float sum_pairs(uint64_t a, uint64_t b) {
+    return (__uint_as_float((uint32_t)a) + __uint_as_float((uint32_t)b)) +
+           (__uint_as_float((uint32_t)(a >> 32)) + __uint_as_float((uint32_t)(b >> 32)));
+}
+#endif
+
 }  // namespace q4dev

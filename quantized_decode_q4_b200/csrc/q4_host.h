@@ -56,14 +56,14 @@ q4_status check_matrix(const q4_matrix* m);
 // multiprocessor count.
 q4_status ensure_device(int* num_sms);
 
-// Batch-1 plan of one launch over `count` GEMVs for a device with `num_sms`
+// CUDA-core plan (1 .. q4b::kMaxTokens tokens) of one launch over `count` GEMVs for a device with `num_sms`
 // multiprocessors: pieces, splits, shared-memory layout, tickets and partial
 // sums (from byte part_base of the workspace). Fills everything except the
 // pointers. *tickets = ticket words used, *ws_end = end of the partial sums.
-q4_status plan_b1(const Shape* sh, int count, int64_t part_base, int num_sms, q4b::Params* P,
+q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_sms, q4b::Params* P,
                   int64_t* tickets, int64_t* ws_end);
 
-// Tensor-core plan (2 <= b <= 16) of one launch; same outputs.
+// Tensor-core plan (q4b::kMaxTokens < b <= 16) of one launch; same outputs.
 q4_status plan_tc(const Shape* sh, int count, int b, int64_t part_base, int num_sms,
                   q4t::Params* P, int64_t* tickets, int64_t* ws_end);
 

@@ -97,19 +97,20 @@ def _groups_of_workloads():
     return sorted(out)
 
 
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
 @pytest.mark.parametrize("num_sms", [148, 132, 160, 7])
-def test_batch1_plans_replay_on_host(num_sms):
+def test_batch1_plans_replay_on_host(num_sms, b):
     """Every byte the batch-1 kernel reads was copied from the right place and its
     lane reads the scale of its own block, every (row, slice) is covered once, the
     shared-memory layout fits two CTAs per SM, split-K scratch stays inside the
     workspace - for every workload shape and group, the edge shapes, and devices
     with other multiprocessor counts."""
     for s in _all_shapes() + EDGE_SHAPES + [(1000, 2080), (3, 992), (4096, 14368)]:
-        assert q4.check_b1([s], num_sms) == 0, (s, num_sms)
+        assert q4.check_b1([s], num_sms, b) == 0, (s, num_sms, b)
     for shapes in _groups_of_workloads():
-        assert q4.check_b1(list(shapes), num_sms) == 0, (shapes, num_sms)
-    assert q4.check_b1([(5, 96), (700, 2080), (3, 4160)], num_sms) == 0
-    assert q4.check_b1([(8, 65536)] * 8, num_sms) == 0
+        assert q4.check_b1(list(shapes), num_sms, b) == 0, (shapes, num_sms, b)
+    assert q4.check_b1([(5, 96), (700, 2080), (3, 4160)], num_sms, b) == 0
+    assert q4.check_b1([(8, 65536)] * 8, num_sms, b) == 0
 
 
 def test_batch1_plans_replay_random_groups():
@@ -121,7 +122,7 @@ def test_batch1_plans_replay_random_groups():
     for _ in range(200):
         shapes = [(int(rng.choice(ns)), 32 * int(rng.choice(kbs)))
                   for _ in range(int(rng.integers(1, 9)))]
-        assert q4.check_b1(shapes) == 0, shapes
+        assert q4.check_b1(shapes, 148, 1 + len(shapes) % 4) == 0, shapes
     rng = np.random.default_rng(7)
     for _ in range(40):
         shapes = [(int(rng.integers(1, 9)), 32 * int(rng.choice([1024, 1500, 2048, 4096])))
