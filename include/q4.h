@@ -132,18 +132,24 @@ q4_status q4_gemv(const q4_matrix* m, const float* x, float* y, void* ws, size_t
                   void* stream);
 
 /* q4_gemv_batched — Y[t] = W X[t] for t < b, 1 <= b <= 16 ("batch 1 to a few
- * tokens"). b = 1 is q4_gemv. For b >= 2 one launch serves all tokens on the
- * tensor cores: the matrix-matrix form of "Llamas on the Web" section 3, the
- * weights dequantised once into on-chip (tensor) memory and reused for every
- * token. Each 32-weight block's codes become (q - 8) in bf16 (exact), each
- * activation x is taken as bf16 parts hi + lo with |x - hi - lo| <= 2^-16 |x|,
- * every block has its own binary32 accumulator and its binary16 scale is
- * applied once: |Y - W X| <= 2^-16 sum |w x| plus binary32 accumulation.
+ * tokens"). b = 1 is q4_gemv. Every b reads each weight once per call, in one
+ * launch for all tokens:
+ *  - 2 <= b <= 4, on the CUDA cores: each code word is unpacked once in
+ *    registers into the exact binary32 values q - 8 ("Llamas on the Web"
+ *    section 3, mat-vec dequantised in registers) and every token multiplies
+ *    them with its own activations; products, block sums and the binary16
+ *    scale in binary32: |Y - W X| within binary32 accumulation.
+ *  - b >= 5, on the tensor cores: the matrix-matrix form of section 3, the
+ *    weights dequantised once into on-chip (tensor) memory and reused for every
+ *    token. Each 32-weight block's codes become (q - 8) in bf16 (exact), each
+ *    activation x is taken as bf16 parts hi + lo with |x - hi - lo| <= 2^-16 |x|,
+ *    every block has its own binary32 accumulator and its binary16 scale is
+ *    applied once: |Y - W X| <= 2^-16 sum |w x| plus binary32 accumulation.
  *   X : device, binary32 [b][m->k] row-major, 16-byte aligned.
  *   Y : device, binary32 [b][m->n] row-major, 16-byte aligned.
  *   ws: as for q4_gemv with q4_workspace_bytes(n, k, b).
  * Errors: as q4_gemv, plus Q4_ERR_UNSUPPORTED for b outside 1..16 and
- * Q4_ERR_INVALID_ARG for n or (n / 128) * (k / 32) at or above 2^31 when b >= 2. */
+ * Q4_ERR_INVALID_ARG for n or (n / 128) * (k / 32) at or above 2^31 when b >= 5. */
 q4_status q4_gemv_batched(const q4_matrix* m, const float* X, int b, float* Y, void* ws,
                           size_t ws_bytes, void* stream);
 
