@@ -1,4 +1,4 @@
-// Batched (2..16 tokens) Q4_0 decode GEMV on the sm_100a tensor cores.
+// Batched (5..16 tokens) Q4_0 decode GEMV on the sm_100a tensor cores.
 //
 // "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
 // section 3 "Dequantizzazione Integrata": for a matrix-matrix product the
@@ -634,7 +634,8 @@ cudaError_t launch_one(const q4t::Params& P, bool pdl, cudaStream_t stream) {
 }  // namespace
 
 // Token count a launch is compiled for: the smallest of 2, 4, 8, 16 >= b.
-int tc_tokens(int b) { return b <= 2 ? 2 : b <= 4 ? 4 : b <= 8 ? 8 : 16; }
+// Token columns of the compiled kernels (up to four tokens take the CUDA-core kernel).
+int tc_tokens(int b) { return b <= 8 ? 8 : 16; }
 
 // Tensor maps of one GEMV for b tokens (rows and columns past the ends read as
 // zero): code plane uint8 [n][k/2], box 128 B x 128 rows with the 128-byte
@@ -663,16 +664,12 @@ cudaError_t encode_tc_maps(q4t::Maps* maps, int32_t* d_box, const uint8_t* qs, c
 
 cudaError_t setup_tc_kernels(int optin_smem) {
     cudaError_t e;
-    if ((e = setup_one<2>(optin_smem)) != cudaSuccess) return e;
-    if ((e = setup_one<4>(optin_smem)) != cudaSuccess) return e;
     if ((e = setup_one<8>(optin_smem)) != cudaSuccess) return e;
     return setup_one<16>(optin_smem);
 }
 
 cudaError_t launch_tc(const q4t::Params& P, bool pdl, cudaStream_t stream) {
     switch (tc_tokens(P.b)) {
-        case 2: return launch_one<2>(P, pdl, stream);
-        case 4: return launch_one<4>(P, pdl, stream);
         case 8: return launch_one<8>(P, pdl, stream);
         default: return launch_one<16>(P, pdl, stream);
     }
