@@ -137,7 +137,9 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
         G.piece_begin = (int32_t)pb;
         G.cps = (int32_t)cps[i];
         pb += G.splits * cps[i];
-        const int64_t rows_max = ceil_div(sh[i].n, cps[i]);
+        int64_t rows_max = 0;  // the first (widest) row range
+        for (int64_t j = 0; j < cps[i]; ++j)
+            rows_max = std::max(rows_max, q4b::range_start(sh[i].n, cps[i], j + 1) - q4b::range_start(sh[i].n, cps[i], j));
         red_floats = std::max<int64_t>(red_floats,
                                        ceil_div(rows_max, q4b::kTileRows) * q4b::kTileRows * G.slices_per_split * b);
     }

@@ -3,11 +3,11 @@
 //
 // A launch covers one dependency group (up to Q4_MAX_GROUP GEMVs). Its work is
 // cut into pieces, one per CTA: GEMV g owns pieces [piece_begin, piece_begin +
-// splits * cps), piece piece_begin + split * cps + j being rows
-// [n j / cps, n (j + 1) / cps) of K split `split`. K is split into ranges of a few
-// slices of 32 blocks (1024 weights, one block per lane; one slice per split by
-// default), so that the activations a piece stages stay small next to its
-// weights. Within a piece, K is walked in slices and rows in tiles of 8: unit
+// splits * cps), piece piece_begin + j * splits + split being row range j of
+// the cps ranges of K split `split` (see piece_of). K is split into ranges of at
+// most a few slices of 32 blocks (1024 weights, one block per lane), so that the
+// activations a piece stages stay small next to its weights. Within a piece, K
+// is walked in slices and rows in tiles of 8: unit
 // u = t * S + s is tile t, slice s of the piece's S slices (tile-major, so a
 // consumer warp that takes every 8th unit keeps one slice when S divides 8).
 //
@@ -143,7 +143,23 @@ struct Params {
     uint32_t* ws;
 };
 
-// Piece c of a launch.
+// Row ranges of a GEMV's pieces may be skewed (a build parameter; equal by
+// default, which measured fastest): row range j of `cps` has weight
+// 1 + a (1 - (2 j + 1) / cps), a = kRowSkew / 16, and its first row is
+// n (j + a (j - j^2 / cps)) / cps (0 for j = 0, n for j = cps).
+#ifndef Q4B_ROW_SKEW
+#define Q4B_ROW_SKEW 0
+#endif
+constexpr int kRowSkew = Q4B_ROW_SKEW;  // sixteenths
+static_assert(kRowSkew > -16 && kRowSkew < 16, "row skew below 1 in magnitude");
+
+Q4B_HD int64_t range_start(int64_t n, int64_t cps, int64_t j) {
+    return n * (16 * j * cps + kRowSkew * j * (cps - j)) / (16 * cps * cps);
+}
+
+// Piece c of a launch. A GEMV's pieces are ordered row range first: piece
+// piece_begin + j * splits + split covers row range j of K split `split`, so the
+// pieces of one row range (one ticket) start together.
 template <class PP>
 Q4B_HD Piece piece_of(const PP& P, int c) {
     int g = 0;
@@ -152,11 +168,11 @@ Q4B_HD Piece piece_of(const PP& P, int c) {
     const int local = c - G.piece_begin;
     Piece p;
     p.g = g;
-    p.split = local / G.cps;
-    const int j = local - p.split * G.cps;
+    const int j = local / G.splits;
+    p.split = local - j * G.splits;
     p.j = j;
-    p.r0 = (int32_t)(G.n * j / G.cps);
-    p.r1 = (int32_t)(G.n * (j + 1) / G.cps);
+    p.r0 = (int32_t)range_start(G.n, G.cps, j);
+    p.r1 = (int32_t)range_start(G.n, G.cps, j + 1);
     return p;
 }
 

@@ -82,7 +82,7 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int 
         // shared only with the pieces of the same rows in the other splits
         if (pc.j < 0 || pc.j >= G.cps || pc.j >= G.n) return 8;
         if (G.splits > 1) {
-            const Piece q0 = piece_of(P, G.piece_begin + pc.j);
+            const Piece q0 = piece_of(P, G.piece_begin + pc.j * G.splits);
             if (q0.split != 0 || q0.j != pc.j || q0.r0 != pc.r0 || q0.r1 != pc.r1) return 8;
         }
         int s0 = 0, S = 0;
