@@ -22,18 +22,10 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
-// 32-block slices of K per batch-1 piece, at most (at most 14: the staged
-// activations of a piece must leave room for the weight ring). Fewer slices mean
-// less activation staging per piece but a split-K reduction at the end.
-#ifndef Q4B_PIECE_SLICES
-#define Q4B_PIECE_SLICES 4
-#endif
-constexpr int kPieceSlices = Q4B_PIECE_SLICES;
 // Pieces the K-split rule for narrow groups aims at (two per multiprocessor of a
 // B200). A constant, not the device's count, so that workspace sizes do not
 // depend on the device.
 constexpr int64_t kSplitPieces = 296;
-static_assert(kPieceSlices >= 1 && kPieceSlices <= q4b::kMaxSlices, "slices per piece");
 // Shared-memory bytes a piece's per-(row, slice) partial sums may take: more
 // rows per piece give it more pieces (CTAs).
 constexpr int64_t kRedPref = 8192;
@@ -89,10 +81,10 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
         q4b::Desc& G = P->g[i];
         const int64_t nb = sh[i].k / Q4_QK;
         const int64_t nsl = ceil_div(nb, q4b::kSliceBlocks);
-        // K in splits of kPieceSlices slices: a piece stages only the activations
+        // K in splits of q4b::kPieceSlices slices: a piece stages only the activations
         // of its own slices (read by every piece of the split), so short K-ranges
         // keep that traffic small next to the piece's weights
-        const int64_t s0 = std::max(ceil_div(nsl, kPieceSlices), std::min(nsl, want));
+        const int64_t s0 = std::max(ceil_div(nsl, q4b::kPieceSlices), std::min(nsl, want));
         const int64_t sps = ceil_div(nsl, s0);
         const int64_t splits = ceil_div(nsl, sps);
         G.n = sh[i].n;

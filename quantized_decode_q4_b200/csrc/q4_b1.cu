@@ -63,9 +63,9 @@ __device__ __forceinline__ float half_bits_f32(uint32_t h) {
 // block; the block's largest |x|, digit sums and flag are reduced over them with
 // shuffles.
 __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
-    float4 v[q4b::kMaxSlices];
+    float4 v[q4b::kPieceSlices];
 #pragma unroll
-    for (int m = 0; m < q4b::kMaxSlices; ++m) {
+    for (int m = 0; m < q4b::kPieceSlices; ++m) {
         const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
         const int s = jl >> 5, jb = jl & 31;
@@ -75,7 +75,7 @@ __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8
                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 #pragma unroll
-    for (int m = 0; m < q4b::kMaxSlices; ++m) {
+    for (int m = 0; m < q4b::kPieceSlices; ++m) {
         if (m >= S) break;
         const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;

@@ -78,8 +78,14 @@ constexpr int kXChunks = kXBlockBytes / 16;   // 16-byte chunks per staged block
 constexpr int kXSliceBytes = kSliceBlocks * kXBlockBytes;
 constexpr int kXFSliceBytes = kSliceBlocks * 128;  // one token's slice in binary32 (2..4 tokens)
 // Slices of one piece, at most (its activations are staged whole, and must leave
-// room for the weight ring).
+// room for the weight ring). Fewer slices mean less activation staging per piece
+// but a split-K reduction at the end; four measured fastest.
+#ifndef Q4B_PIECE_SLICES
+#define Q4B_PIECE_SLICES 4
+#endif
+constexpr int kPieceSlices = Q4B_PIECE_SLICES;
 constexpr int kMaxSlices = 14;
+static_assert(kPieceSlices >= 1 && kPieceSlices <= kMaxSlices, "slices per piece");
 // Ring slots: a multiple of kWarps, so that every unit routed to a slot
 // (u = slot mod slots) belongs to the same warp, which both requests and waits
 // for it: the warp is never more than one phase ahead of the slot's barrier,

@@ -87,7 +87,7 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int 
         }
         int s0 = 0, S = 0;
         piece_slices(G, pc.split, &s0, &S);
-        if (S < 1 || s0 + S > G.nslices) return 9;
+        if (S < 1 || S > kPieceSlices || s0 + S > G.nslices) return 9;  // staging holds kPieceSlices
         if (b == 1) {
             if ((uint32_t)S * kXSliceBytes > P.x_bytes) return 10;
             if (xchunk_offset(S - 1, kXChunks - 1, kSliceBlocks - 1) + 16 > P.x_bytes) return 10;
