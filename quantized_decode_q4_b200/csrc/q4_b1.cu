@@ -3,7 +3,7 @@
 // "Llamas on the Web" (gist.science technical summary of arXiv 2605.20706),
 // section 3 "Dequantizzazione Integrata": the decode mat-vec dequantises in
 // registers; no dequantised weight is ever written to memory. The work split is
-// described in q4_b1_plan.h. Per CTA (8 warps, two CTAs per SM):
+// described in q4_b1_plan.h. Per CTA (8 warps; two CTAs fit one SM):
 //  * the piece's units (8 rows x 32 blocks: 4 KB of codes and their binary16
 //    scales) stream from HBM into a ring of shared-memory slots as 2-D tensor
 //    loads on the TMA engine, each completing on its slot's mbarrier. The first

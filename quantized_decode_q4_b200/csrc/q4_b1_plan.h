@@ -18,11 +18,14 @@
 // stride is not a multiple of 16 bytes is copied row by row instead); the first
 // `slots` units are requested at kernel entry, and each warp, once it has read
 // unit u, requests unit u + slots into the slot it just freed. Warps multiply
-// units with the piece's activations (quantised once per piece into shared
-// memory) and write per-(row, slice) partial sums to shared memory; after the last unit the CTA adds each row's slices in slice
-// order and stores y (or a split-K partial; the last piece of a row range to
-// arrive adds the range's partials up in split order). Two CTAs of consecutive launches fit one SM, so a
-// launch streams its weights in while the previous one finishes.
+// units with the piece's activations (staged once per piece in shared memory)
+// and write per-(row, slice) partial sums to shared memory; after the last unit
+// the CTA adds each row's slices in slice order and stores y (or a split-K
+// partial; the last piece of a row range to arrive adds the range's partials up
+// in split order). For 1 and 2 tokens a launch has one piece per SM although two
+// CTAs fit: the SM's other CTA slot takes the next launch's CTA, which streams
+// its first units in while this one computes (measured 6% faster than two pieces
+// per SM for one token).
 #pragma once
 
 #include <cuda.h>
@@ -90,9 +93,9 @@ static_assert(kPieceSlices >= 1 && kPieceSlices <= kMaxSlices, "slices per piece
 // (u = slot mod slots) belongs to the same warp, which both requests and waits
 // for it: the warp is never more than one phase ahead of the slot's barrier,
 // which a parity wait requires.
-// Pieces (CTAs) of one launch per multiprocessor: as many as fit at once.
+// Pieces (CTAs) of one launch per multiprocessor (at most as many as fit at once).
 #ifndef Q4B_PIECES_PER_SM
-#define Q4B_PIECES_PER_SM 2
+#define Q4B_PIECES_PER_SM 1
 #endif
 Q4B_HD_CONST int pieces_per_sm(int b) { return ctas_per_sm(b) == 2 ? Q4B_PIECES_PER_SM : 1; }
 Q4B_HD_CONST int max_slots(int b) { return 48 / ctas_per_sm(b) / kWarps * kWarps; }
