@@ -91,7 +91,7 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
         G.nb = (int32_t)nb;
         G.nslices = (int32_t)nsl;
         G.splits = (int32_t)splits;
-        G.slices_per_split = (int32_t)sps;
+        G.slices_per_split = (int32_t)ceil_div(nsl, splits);
         G.d_map = nb % 8 == 0 ? 1 : 0;
         if (splits > 1) {
             G.ticket_off = kHeaderBytes / 4 + tick;
@@ -99,12 +99,12 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
             G.part_off = part / 4;
             part += round_up(splits * b * sh[i].n * 4, 256);  // [splits][b][n]
         }
-        max_slices = std::max<int>(max_slices, (int)sps);
+        max_slices = std::max<int>(max_slices, G.slices_per_split);
         // rows of one piece: its per-(token, row, slice) partial sums stay within kRedPref
         const int64_t max_rows = std::max<int64_t>(
             q4b::kTileRows, kRedPref / 4 / sps / b / q4b::kTileRows * q4b::kTileRows);
         cps[i] = std::min<int64_t>(sh[i].n, ceil_div(sh[i].n, max_rows));
-        wsplit[i] = std::min<int64_t>(nb, sps * q4b::kSliceBlocks);  // blocks of a split
+        wsplit[i] = std::min<int64_t>(nb, G.slices_per_split * q4b::kSliceBlocks);  // blocks of a split
     }
     if (kHeaderBytes + 4 * tick > part_base) return Q4_ERR_INVALID_ARG;
     // spare CTAs (up to q4b::pieces_per_sm(b) per multiprocessor): to the GEMV whose

@@ -120,7 +120,7 @@ struct Desc {
     int32_t nb;                // k / 32
     int32_t nslices;           // ceil(nb / 32)
     int32_t splits;            // K splits across CTAs
-    int32_t slices_per_split;
+    int32_t slices_per_split;  // slices of the widest split
     int32_t piece_begin;       // first piece (CTA) of this GEMV
     int32_t cps;               // pieces (CTAs) per split
     int32_t d_map;             // 1: scales loaded by the tensor map (row stride % 16 == 0)
@@ -193,10 +193,11 @@ Q4B_HD uint32_t x_offset(const Params& P) { return (uint32_t)kBarBytes + P.red_b
 Q4B_HD uint32_t ring_offset(const Params& P) { return (uint32_t)kBarBytes + P.red_bytes + P.x_bytes; }
 
 // Slices of a piece: first global slice and count.
+// Splits cover nslices * split / splits .. nslices * (split + 1) / splits: as
+// even as whole slices allow (at most slices_per_split = ceil(nslices / splits)).
 Q4B_HD void piece_slices(const Desc& G, int split, int* s0, int* S) {
-    *s0 = split * G.slices_per_split;
-    const int rest = G.nslices - *s0;
-    *S = rest < G.slices_per_split ? rest : G.slices_per_split;
+    *s0 = (int)((int64_t)G.nslices * split / G.splits);
+    *S = (int)((int64_t)G.nslices * (split + 1) / G.splits) - *s0;
 }
 
 // Blocks of global slice gs (32, or fewer in the last slice).
