@@ -379,36 +379,27 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::ctas_per_sm(B))
                     sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
                                 : q4b::scale_offset(G, pc, t, gs, r, lane)));
                 const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-                uint64_t acc[B][q4b::kTokenChains];
+                uint64_t acc[B][2];  // two chains per token: even and odd words
 #pragma unroll
-                for (int tk = 0; tk < B; ++tk)
-#pragma unroll
-                    for (int c = 0; c < q4b::kTokenChains; ++c) acc[tk][c] = 0ull;
+                for (int tk = 0; tk < B; ++tk) acc[tk][0] = acc[tk][1] = 0ull;
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     uint64_t pr[4];
                     code_pairs(words[w], kc, pr);
 #pragma unroll
                     for (int tk = 0; tk < B; ++tk) {
-                        uint64_t a = acc[tk][w % q4b::kTokenChains];
+                        uint64_t a = acc[tk][w & 1];
                         a = ffma2(pr[0], xp[tk][2 * w], a);
                         a = ffma2(pr[1], xp[tk][2 * w + 1], a);
                         a = ffma2(pr[2], xp[tk][2 * w + 8], a);
                         a = ffma2(pr[3], xp[tk][2 * w + 9], a);
-                        acc[tk][w % q4b::kTokenChains] = a;
+                        acc[tk][w & 1] = a;
                     }
                 }
                 const float d = half_bits_f32(dh);
                 const bool live = whole || (lane < bs && r < nr);
 #pragma unroll
-                for (int tk = 0; tk < B; ++tk) {
-                    uint64_t a0 = acc[tk][0], a1 = acc[tk][1];
-                    if constexpr (q4b::kTokenChains == 4) {
-                        a0 = fadd2(a0, acc[tk][2]);
-                        a1 = fadd2(a1, acc[tk][3]);
-                    }
-                    v[tk][r] = live ? d * sum_pairs(a0, a1) : 0.0f;
-                }
+                for (int tk = 0; tk < B; ++tk) v[tk][r] = live ? d * sum_pairs(acc[tk][0], acc[tk][1]) : 0.0f;
             }
         } else if (!lx.flagged) {
             const float ls = lx.scale;

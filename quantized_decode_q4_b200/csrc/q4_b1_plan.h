@@ -58,18 +58,9 @@ constexpr int kCtasPerSm = Q4B_CTAS_PER_SM;
 #define Q4B_MAX_TOKENS 4
 #endif
 constexpr int kMaxTokens = Q4B_MAX_TOKENS;
-#ifndef Q4B_CTAS_PER_SM_B2
-#define Q4B_CTAS_PER_SM_B2 Q4B_CTAS_PER_SM
-#endif
-// Accumulator chains per token and row of the 2..4-token path (2 or 4).
-#ifndef Q4B_TOKEN_CHAINS
-#define Q4B_TOKEN_CHAINS 2
-#endif
-constexpr int kTokenChains = Q4B_TOKEN_CHAINS;
-static_assert(kTokenChains == 2 || kTokenChains == 4, "accumulator chains");
 // CTAs per SM for b tokens: three and four tokens keep 32 b activation values per
 // lane in registers, which takes the register file of a whole SM.
-Q4B_HD_CONST int ctas_per_sm(int b) { return b == 1 ? kCtasPerSm : (b == 2 ? Q4B_CTAS_PER_SM_B2 : 1); }
+Q4B_HD_CONST int ctas_per_sm(int b) { return b <= 2 ? kCtasPerSm : 1; }
 constexpr int kTileRows = 8;                  // rows per unit
 constexpr int kSliceBlocks = 32;              // blocks per unit (one per lane)
 constexpr int kSlotQs = kTileRows * kSliceBlocks * 16;  // code bytes of a unit
@@ -152,19 +143,8 @@ struct Params {
     uint32_t* ws;
 };
 
-// Row ranges of a GEMV's pieces may be skewed (a build parameter; equal by
-// default, which measured fastest): row range j of `cps` has weight
-// 1 + a (1 - (2 j + 1) / cps), a = kRowSkew / 16, and its first row is
-// n (j + a (j - j^2 / cps)) / cps (0 for j = 0, n for j = cps).
-#ifndef Q4B_ROW_SKEW
-#define Q4B_ROW_SKEW 0
-#endif
-constexpr int kRowSkew = Q4B_ROW_SKEW;  // sixteenths
-static_assert(kRowSkew > -16 && kRowSkew < 16, "row skew below 1 in magnitude");
-
-Q4B_HD int64_t range_start(int64_t n, int64_t cps, int64_t j) {
-    return n * (16 * j * cps + kRowSkew * j * (cps - j)) / (16 * cps * cps);
-}
+// First row of row range j of the cps equal ranges of n rows.
+Q4B_HD int64_t range_start(int64_t n, int64_t cps, int64_t j) { return n * j / cps; }
 
 // Piece c of a launch. A GEMV's pieces are ordered row range first: piece
 // piece_begin + j * splits + split covers row range j of K split `split`, so the

@@ -307,12 +307,6 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
     return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
 }
