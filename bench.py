@@ -356,8 +356,7 @@ def measure_configs(peak: float, shared=None, min_steps: int = 200, max_seconds:
                 "q4_bytes_per_step": step.q4_bytes, "launches_per_step": step.launches,
                 "weight_copies": r, "steps_timed": reps * r,
                 "l2": f"cold: {r} weight copies, {r * step.q4_bytes / 1e6:.0f} MB in turn",
-                "kernel": ("q4k::stack_b1_kernel" if b == 1 else "q4k::gemv_b1_kernel"
-                           if b <= SMALL_BATCH else "q4k::gemv_tc_kernel")}
+                "kernel": "q4k::gemv_b1_kernel" if b <= SMALL_BATCH else "q4k::gemv_tc_kernel"}
             del g, stacks, step
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
@@ -555,13 +554,8 @@ def main():
                           "(2^-16 relative), binary32 accumulators and sums"),
                 "gemvs_per_step": len(workload.gemvs), "q4_bytes_per_step": q4_bytes,
                 "weights": "Q4_0 planes (4.5 bits/weight), binary32 activations and sums",
-                "launch": ((f"one CUDA graph per step: {step.launches} PDL-chained launches of the "
-                            "persistent stack kernel (one CTA per SM through consecutive groups)"
-                            if args.batch == 1 else
-                            "one CUDA graph per step of PDL-chained group launches")
-                           if graph is not None else
-                           (f"{step.launches} PDL-chained launches of the persistent stack kernel"
-                            if args.batch == 1 else "PDL-chained group launches")),
+                "launch": ("one CUDA graph per step of PDL-chained group launches"
+                           if graph is not None else "PDL-chained group launches"),
                 "l2": (f"no flush: the weights of one step ({q4_bytes / 1e9:.2f} GB) are "
                        f"{q4_bytes / L2_BYTES:.0f}x the 126 MB L2"
                        if q4_bytes > 4 * L2_BYTES else
@@ -574,8 +568,7 @@ def main():
             "roofline": {
                 "bound": "hbm", "achieved": per_gpu_alg, "peak": peak, "unit": "GB/s",
                 "frac": per_gpu_alg / peak, "traffic": traffic,
-                "kernel": ("q4k::stack_b1_kernel" if args.batch == 1 else
-                           "q4k::gemv_b1_kernel" if args.batch <= SMALL_BATCH else
+                "kernel": ("q4k::gemv_b1_kernel" if args.batch <= SMALL_BATCH else
                            "q4k::gemv_tc_kernel"),
                 "peak_source": peak_src,
                 "note": ("achieved = algorithmic bytes of a step (Q4_0 weights + x + y) / step "

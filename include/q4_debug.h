@@ -30,21 +30,6 @@ extern "C" {
  * of the first failed check (see q4_debug.cu). */
 int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int num_sms);
 
-/* Plan a one-token q4_layer_stack of `count` GEMVs (shapes n[i] x k[i], group
- * numbers group[i]) as the library would on a device with `num_sms`
- * multiprocessors, for its persistent stack kernel, and replay it on the host:
- * groups split into launches that fit the kernel's parameters (each as long as
- * possible), every group planned as its own batch-1 launch would be, shared
- * memory inside the budget, at most one CTA per multiprocessor, completion counts
- * after the tickets and before the partial sums, and, for every CTA and warp, the
- * sequence of units it requests walked exactly as the device walks it: each unit
- * a warp reads is the one it requested into that slot, in the same order, every
- * request is read, and every unit of every piece is read exactly once.
- * *launches (if not null) = launches of the stack. Returns 0 when every check
- * holds, otherwise the number of the first failed check (see q4_debug.cu). */
-int q4_debug_check_stack(const int64_t* n, const int64_t* k, const int* group, int count, int num_sms,
-                         int64_t* launches);
-
 /* Summary of the CUDA-core plan above for a 148-multiprocessor B200 (1 <= b <= 4):
  * out[0] = CTAs (pieces), out[1] = dynamic shared memory bytes per CTA,
  * out[2] = workspace bytes, out[3] = weight ring slots, out[4 + i] = K splits of

@@ -77,8 +77,6 @@ def lib():
             "q4_launch_count": ([], c.c_uint64),
             "q4_last_cuda_error": ([], c.c_char_p),
             "q4_debug_check_b1": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int, c.c_int], c.c_int),
-            "q4_debug_check_stack": ([c.POINTER(i64), c.POINTER(i64), c.POINTER(c.c_int), c.c_int, c.c_int,
-                                      c.POINTER(i64)], c.c_int),
             "q4_gemv_noalloc": ([mp, vp, vp, vp], c.c_int),
             "q4_noalloc_status": ([vp], c.c_int),
             "q4_debug_plan_info": ([c.POINTER(i64), c.POINTER(i64), c.c_int, c.c_int,
@@ -316,17 +314,6 @@ def check_b1(shapes, num_sms: int = 148, b: int = 1) -> int:
     n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
     k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
     return lib().q4_debug_check_b1(n, k, len(shapes), b, num_sms)
-
-
-def check_stack(shapes, groups, num_sms: int = 148):
-    """Host replay of the one-token persistent stack plan: (status, launches);
-    status 0 when every check holds."""
-    n = (ctypes.c_int64 * len(shapes))(*[s[0] for s in shapes])
-    k = (ctypes.c_int64 * len(shapes))(*[s[1] for s in shapes])
-    g = (ctypes.c_int * len(shapes))(*groups)
-    nl = ctypes.c_int64(0)
-    st = lib().q4_debug_check_stack(n, k, g, len(shapes), num_sms, ctypes.byref(nl))
-    return st, nl.value
 
 
 def plan_info(shapes, b: int = 1) -> dict:

@@ -9,7 +9,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <memory>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -150,71 +149,6 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
     P->slots = (int32_t)slots;
     *tickets = tick;
     *ws_end = part;
-    return Q4_OK;
-}
-
-// ---------------------------------------------------------------------------
-// persistent batch-1 stack plan
-// ---------------------------------------------------------------------------
-
-// Pieces of group g for one token (0 if it cannot be planned).
-int group_pieces(const Shape* sh, const std::pair<int, int>& g, int num_sms) {
-    q4b::Params P;
-    int64_t t = 0, end = 0;
-    if (plan_b1(sh + g.first, g.second - g.first, 1, 0x40000000LL, num_sms, &P, &t, &end) != Q4_OK) return 0;
-    return P.npieces;
-}
-
-void stack_chunk(const Shape* sh, const std::vector<std::pair<int, int>>& groups, int g0, int num_sms, int* g1,
-                 bool* alone) {
-    *alone = group_pieces(sh, groups[g0], num_sms) > num_sms;
-    if (*alone) {
-        *g1 = g0 + 1;
-        return;
-    }
-    int g = g0, gemvs = 0;
-    while (g < (int)groups.size() && g - g0 < q4s::kStackGroups &&
-           gemvs + (groups[g].second - groups[g].first) <= q4s::kStackGemvs &&
-           group_pieces(sh, groups[g], num_sms) <= num_sms) {
-        gemvs += groups[g].second - groups[g].first;
-        ++g;
-    }
-    *g1 = g;
-}
-
-q4_status plan_stack(const Shape* sh, const std::vector<std::pair<int, int>>& groups, int g0, int g1,
-                     int64_t part_base, int64_t count_word, int num_sms, q4s::Params* P, int* grid) {
-    if (g1 <= g0 || g1 - g0 > q4s::kStackGroups) return Q4_ERR_INVALID_ARG;
-    std::memset(P, 0, sizeof *P);
-    uint32_t red = 0, xb = 0;
-    int gm = 0, maxp = 0;
-    for (int gi = g0; gi < g1; ++gi) {
-        const int first = groups[gi].first, count = groups[gi].second - first;
-        if (gm + count > q4s::kStackGemvs) return Q4_ERR_INVALID_ARG;
-        q4b::Params G;
-        int64_t t = 0, end = 0;
-        q4_status s = plan_b1(sh + first, count, 1, part_base, num_sms, &G, &t, &end);
-        if (s != Q4_OK) return s;
-        q4s::Group& gr = P->grp[gi - g0];
-        gr.first = gm;
-        gr.count = count;
-        gr.npieces = G.npieces;
-        gr.counter = (int32_t)(count_word + gi);
-        for (int i = 0; i < count; ++i) P->gemv[gm + i].desc = G.g[i];
-        gm += count;
-        red = std::max(red, G.red_bytes);
-        xb = std::max(xb, G.x_bytes);
-        maxp = std::max(maxp, G.npieces);
-    }
-    P->ngroups = g1 - g0;
-    P->red_bytes = red;
-    P->x_bytes = xb;
-    const int64_t room = (int64_t)q4s::kSmemBudget - q4s::kBarBytes - red - xb;
-    const int64_t slots = std::min<int64_t>(room / q4b::kSlotBytes, q4s::kMaxSlots) / q4s::kSWarps * q4s::kSWarps;
-    if (slots < q4s::kSWarps) return Q4_ERR_UNSUPPORTED;
-    P->slots = (int32_t)slots;
-    if (maxp > num_sms) return Q4_ERR_UNSUPPORTED;  // every CTA must be resident at once
-    *grid = maxp;
     return Q4_OK;
 }
 
@@ -458,10 +392,8 @@ q4_status stack_args(const q4_stack* s, int b, std::vector<std::pair<int, int>>*
 
 // Validate a stack; returns the ticket region shared by all groups and the
 // workspace bytes needed.
-// For one token the persistent stack kernel also keeps one completion count
-// per group, after the tickets (*count_word, when given, is the first).
 q4_status stack_check(const q4_stack* s, int b, int num_sms, std::vector<std::pair<int, int>>* groups,
-                      int64_t* tickets, size_t* need, int64_t* count_word = nullptr) {
+                      int64_t* tickets, size_t* need) {
     q4_status st = stack_groups(s, groups);
     if (st != Q4_OK) return st;
     int64_t tmax = 0, pmax = 0;
@@ -474,66 +406,12 @@ q4_status stack_check(const q4_stack* s, int b, int num_sms, std::vector<std::pa
         tmax = std::max(tmax, t);
         pmax = std::max(pmax, p);
     }
-    if (count_word) *count_word = kHeaderBytes / 4 + tmax;
-    if (b == 1) tmax += (int64_t)groups->size();
     *tickets = tmax;
     *need = (size_t)(part_base_for(tmax) + pmax);
     return Q4_OK;
 }
 
 }  // namespace
-
-// Enqueue a one-token stack as launches of the persistent stack kernel, each
-// over as many consecutive groups as its parameters hold.
-q4_status launch_stack(const q4_stack* s, const std::vector<std::pair<int, int>>& groups, void* ws,
-                       int64_t part_base, int64_t count_word, int num_sms, cudaStream_t stream) {
-    std::vector<Shape> sh((size_t)s->count);
-    for (int i = 0; i < s->count; ++i) sh[i] = {s->mats[i].n, s->mats[i].k};
-    std::unique_ptr<q4s::Params> P(new (std::nothrow) q4s::Params);
-    if (!P) return Q4_ERR_INVALID_ARG;
-    bool first = true;
-    for (int g0 = 0; g0 < (int)groups.size();) {
-        int g1 = g0;
-        bool alone = false;
-        stack_chunk(sh.data(), groups, g0, num_sms, &g1, &alone);
-        if (alone) {
-            // more pieces than multiprocessors: the one-group kernel, whose CTAs
-            // never wait for one another
-            GemvCall calls[Q4_MAX_GROUP];
-            for (int i = groups[g0].first; i < groups[g0].second; ++i)
-                calls[i - groups[g0].first] = {s->mats[i], s->x[i], s->y[i]};
-            q4_status st = launch_group(calls, groups[g0].second - groups[g0].first, 1, ws, part_base, num_sms,
-                                        !first, stream);
-            if (st != Q4_OK) return st;
-            first = false;
-            g0 = g1;
-            continue;
-        }
-        int grid = 0;
-        q4_status st = plan_stack(sh.data(), groups, g0, g1, part_base, count_word, num_sms, P.get(), &grid);
-        if (st != Q4_OK) return st;
-        for (int gi = g0; gi < g1; ++gi) {
-            const q4s::Group& gr = P->grp[gi - g0];
-            for (int i = 0; i < gr.count; ++i) {
-                const int src = groups[gi].first + i;
-                q4s::Gemv& M = P->gemv[gr.first + i];
-                M.desc.qs = s->mats[src].qs;
-                M.desc.d = s->mats[src].d;
-                M.desc.x = s->x[src];
-                M.desc.y = s->y[src];
-                if (cuda_failed(q4k::encode_b1_maps(&M.qs_map, &M.d_map, &M.desc.d_map, s->mats[src].qs,
-                                                    s->mats[src].d, s->mats[src].n, s->mats[src].k)))
-                    return Q4_ERR_CUDA;
-            }
-        }
-        P->ws = static_cast<uint32_t*>(ws);
-        if (cuda_failed(q4k::launch_stack_b1(*P, grid, !first, stream))) return Q4_ERR_CUDA;
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        first = false;
-        g0 = g1;
-    }
-    return Q4_OK;
-}
 
 struct q4_graph_s {
     cudaGraph_t graph;
@@ -658,14 +536,13 @@ q4_status q4_layer_stack(const q4_stack* s, int b, void* ws, size_t ws_bytes, vo
     if (!aligned(ws, 256)) return Q4_ERR_MISALIGNED;
     int num_sms = 0;
     if ((st = ensure_device(&num_sms)) != Q4_OK) return st;
-    int64_t tickets = 0, count_word = 0;
+    int64_t tickets = 0;
     size_t need = 0;
-    if ((st = stack_check(s, b, num_sms, &groups, &tickets, &need, &count_word)) != Q4_OK) return st;
+    if ((st = stack_check(s, b, num_sms, &groups, &tickets, &need)) != Q4_OK) return st;
     if ((st = check_ws(ws, ws_bytes, need)) != Q4_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if ((st = clear_tickets(ws, tickets, cs)) != Q4_OK) return st;
     const int64_t base = part_base_for(tickets);
-    if (b == 1) return launch_stack(s, groups, ws, base, count_word, num_sms, cs);
     bool first = true;
     for (auto& g : groups) {
         GemvCall calls[Q4_MAX_GROUP];
@@ -699,7 +576,6 @@ q4_status q4_stack_graph_create(const q4_stack* s, int b, void* ws, size_t ws_by
     if (cuda_failed(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal))) return Q4_ERR_CUDA;
     const uint64_t before = g_launches.load();
     q4_status run = q4_layer_stack(s, b, ws, ws_bytes, stream);
-    const uint64_t kernels = g_launches.load() - before;
     g_launches.store(before);  // captured launches do not run now
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(cs, &graph);
@@ -721,7 +597,7 @@ q4_status q4_stack_graph_create(const q4_stack* s, int b, void* ws, size_t ws_by
     }
     g->graph = graph;
     g->exec = exec;
-    g->kernels = kernels;
+    g->kernels = (uint64_t)groups.size();
     *out = g;
     return Q4_OK;
 }

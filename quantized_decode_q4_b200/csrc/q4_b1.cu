@@ -37,7 +37,6 @@
 #include "q4_device.cuh"
 #include "q4_intdot.cuh"
 #include "q4_maps.h"
-#include "q4_stack_plan.h"
 
 using namespace q4dev;
 
@@ -57,34 +56,30 @@ __device__ __forceinline__ float half_bits_f32(uint32_t h) {
     return __half2float(__ushort_as_half((unsigned short)h));
 }
 
-// Quantise the piece's activations (all NT threads): item i of S * 32 * 8 is
-// float4 g = i % 8 of block i / 8 (local slice i / 256), and thread `tid` takes
-// items tid + NT m. All of a thread's loads are issued before any is used (one
-// latency instead of several). Eight consecutive lanes share a block; the
-// block's largest |x|, digit sums and flag are reduced over them with shuffles
-// (a warp's 32 items lie in one slice, so a warp takes a round whole or not at
-// all).
-template <int NT>
+// Quantise the piece's activations (all consumer threads): item i of
+// S * 32 * 8 is float4 g = i % 8 of block i / 8 (local slice (i / 8) / 32), and
+// thread `tid` takes items tid + 256 m, m < S. All of a thread's loads are issued
+// before any is used (one latency instead of S). Eight consecutive lanes share a
+// block; the block's largest |x|, digit sums and flag are reduced over them with
+// shuffles.
 __device__ __forceinline__ void stage_x(const q4b::Desc& G, int s0, int S, uint8_t* xs, int tid) {
-    static_assert((q4b::kPieceSlices * 256) % NT == 0 && NT % 256 == 0, "whole slices per round");
-    constexpr int kRounds = q4b::kPieceSlices * 256 / NT;
-    float4 v[kRounds];
+    float4 v[q4b::kPieceSlices];
 #pragma unroll
-    for (int m = 0; m < kRounds; ++m) {
-        const int i = m * NT + tid;
+    for (int m = 0; m < q4b::kPieceSlices; ++m) {
+        const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
         const int s = jl >> 5, jb = jl & 31;
         const int64_t b = (int64_t)(s0 + s) * q4b::kSliceBlocks + jb;
-        v[m] = (s < S && jb < q4b::slice_blocks(G, s0 + s))
+        v[m] = (m < S && jb < q4b::slice_blocks(G, s0 + s))
                    ? __ldcg(reinterpret_cast<const float4*>(G.x + b * 32) + g)
                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 #pragma unroll
-    for (int m = 0; m < kRounds; ++m) {
-        const int i = m * NT + tid;
+    for (int m = 0; m < q4b::kPieceSlices; ++m) {
+        if (m >= S) break;
+        const int i = m * q4b::kWarps * 32 + tid;
         const int jl = i >> 3, g = i & 7;
         const int s = jl >> 5, jb = jl & 31;
-        if (s >= S) break;
         uint32_t mx = max(max(__float_as_uint(v[m].x) & 0x7FFFFFFFu, __float_as_uint(v[m].y) & 0x7FFFFFFFu),
                           max(__float_as_uint(v[m].z) & 0x7FFFFFFFu, __float_as_uint(v[m].w) & 0x7FFFFFFFu));
 #pragma unroll
@@ -329,7 +324,7 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::ctas_per_sm(B))
     pdl_wait();
     const int tid = threadIdx.x;
     if constexpr (B == 1)
-        stage_x<q4b::kThreads>(G, s0, S, xs, tid);
+        stage_x(G, s0, S, xs, tid);
     else
         stage_xf<B>(G, s0, S, xs, tid);
     consumer_sync();
@@ -520,313 +515,6 @@ __global__ void __launch_bounds__(q4b::kThreads, q4b::ctas_per_sm(B))
     if (tid == 0) *ticket = 0u;
 }
 
-// ---------------------------------------------------------------------------
-// Persistent layer-stack kernel (1 token): one CTA per SM runs its piece of
-// every group of the launch, with one weight ring that streams across groups
-// (q4_stack_plan.h).
-// ---------------------------------------------------------------------------
-
-namespace {
-
-// Longest a CTA waits for an earlier group's completion count. Every piece of
-// the launch is resident at once, so a legitimate wait lasts microseconds.
-constexpr uint64_t kCountLimitNs = 200ull * 1000 * 1000;
-
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Wait until *cnt >= want (thread 0 of a CTA). False when the time limit passes
-// or another CTA has recorded a timeout in the workspace header.
-__device__ bool count_wait(const uint32_t* cnt, uint32_t want, const uint32_t* ws) {
-    if (ld_acquire(cnt) >= want) return true;
-    const uint64_t start = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (ld_acquire(cnt) >= want) return true;
-        if ((i & 15) == 0) {
-            if (*reinterpret_cast<const volatile uint32_t*>(ws) & kTimeoutFlag) return false;
-            if (global_ns() - start > kCountLimitNs) return false;
-        }
-        __nanosleep(32);
-    }
-}
-
-// Request unit (q.t, q.s) of the piece q.p into ring slot `slot` (whole warp;
-// see issue_unit).
-template <bool kDMap>
-__device__ __forceinline__ void issue_stack_unit(const q4s::Params& P, const q4s::Seq& q, int slot,
-                                                 uint8_t* ring, uint64_t* full, int lane, int lane_issue) {
-    const q4s::Gemv& M = P.gemv[q.p.gemv];
-    const int gsl = q.p.s0 + q.s;
-    const int32_t row0 = q.p.r0 + q.t * q4b::kTileRows;
-    uint8_t* dst = ring + (size_t)slot * q4b::kSlotBytes;
-    if (kDMap) {
-        if (lane == lane_issue) {
-            mbar_arrive_expect_tx(full + slot, q4b::kMapCodeBytes + q4b::kMapScaleBytes);
-            tma_load_2d(dst, &M.qs_map, gsl * (q4b::kSliceBlocks * 4), row0, full + slot);
-            tma_load_2d(dst + q4b::kSlotQs, &M.d_map, gsl * q4b::kSliceBlocks, row0, full + slot);
-        }
-        return;
-    }
-    q4b::Piece pp;
-    pp.g = 0;
-    pp.split = q.p.split;
-    pp.j = q.p.j;
-    pp.r0 = q.p.r0;
-    pp.r1 = q.p.r1;
-    q4b::LaneCopy c = q4b::lane_copy(M.desc, pp, q.t, gsl, lane);
-    c.active = c.active && c.scales;
-    const uint32_t bytes = c.active ? c.bytes : 0u;
-    const uint32_t total = __reduce_add_sync(0xffffffffu, bytes) + q4b::kMapCodeBytes;
-    if (lane == lane_issue) {
-        mbar_arrive_expect_tx(full + slot, total);
-        tma_load_2d(dst, &M.qs_map, gsl * (q4b::kSliceBlocks * 4), row0, full + slot);
-    }
-    __syncwarp();
-    if (c.active)
-        bulk_g2s(dst + c.dst, reinterpret_cast<const uint8_t*>(M.desc.d) + c.src_off, c.bytes, full + slot);
-}
-
-}  // namespace
-
-template <bool kDMap>
-__global__ void __launch_bounds__(q4s::kSThreads, 1) stack_b1_kernel(const __grid_constant__ q4s::Params P) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    const int c = blockIdx.x;
-    const int slots = P.slots;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    float* red = reinterpret_cast<float*>(smem + q4s::red_offset());
-    uint8_t* xs = smem + q4s::x_offset(P);
-    uint8_t* ring = smem + q4s::ring_offset(P);
-    __shared__ int abort_flag;
-    __shared__ int last_split;
-
-    if (tid == 0) {
-        for (int i = 0; i < slots; ++i) mbar_init(full + i, 1);
-        abort_flag = 0;
-        mbar_fence_init();
-    }
-    __syncthreads();
-    pdl_launch_dependents();
-
-    // unit v of the CTA's sequence is read by warp v % kSWarps from slot
-    // v % slots; the first `slots` units are requested before any wait
-    q4s::Seq rc;  // the next unit this warp requests (sequence index vr)
-    rc.start(P, c, warp);
-    int vr = warp;
-    for (; rc.valid(P) && vr < slots; vr += q4s::kSWarps) {
-        issue_stack_unit<kDMap>(P, rc, vr, ring, full, lane, (vr / q4s::kSWarps) & 31);
-        rc.advance(P, c);
-    }
-
-    volatile int* abort_v = &abort_flag;
-    const UnpackConsts kc = unpack_consts_default();
-    int v = warp;  // sequence index of the next unit this warp reads
-    int slot = warp;
-    uint32_t phase = 0;
-    int base = 0;  // sequence index of the current group's first unit
-    bool waited_grid = false;
-    for (int gi = 0; gi < P.ngroups; ++gi) {
-        q4s::Piece pc;
-        if (!q4s::piece_of(P, gi, c, &pc)) continue;
-        const q4b::Desc& G = P.gemv[pc.gemv].desc;
-        const int S = pc.S, U = pc.U, nb = G.nb;
-        // x into L2 while the wait runs (a hint; L2 is where results land)
-        if (tid == 32) {
-            const int64_t e0 = (int64_t)pc.s0 * q4b::kSliceBlocks * 32;
-            const int64_t e1 = min((int64_t)(pc.s0 + S) * q4b::kSliceBlocks * 32, (int64_t)nb * 32);
-            bulk_prefetch_l2(G.x + e0, (uint32_t)((e1 - e0) * 4));
-        }
-        if (!waited_grid) {
-            pdl_wait();
-            waited_grid = true;
-        }
-        if (gi > 0) {
-            if (tid == 0) {
-                const q4s::Group& Gp = P.grp[gi - 1];
-                if (!count_wait(P.ws + Gp.counter, (uint32_t)Gp.npieces + P.count_extra, P.ws)) {
-                    atomicOr(P.ws, kTimeoutFlag);
-                    abort_flag = 1;
-                }
-            }
-            __syncthreads();
-            if (*abort_v) break;
-        }
-        stage_x<q4s::kSThreads>(G, pc.s0, S, xs, tid);
-        __syncthreads();
-
-        // this warp's units of the group: local u = v - base, stepping kSWarps
-        Cursor cu;
-        cu.set(v - base, S);
-        const int dt = q4s::kSWarps / S, ds = q4s::kSWarps - dt * S;
-        int cur = -1;
-        LaneX lx;
-        for (; v < base + U; v += q4s::kSWarps) {
-            if (*abort_v) break;
-            const int t = cu.t, s = cu.s;
-            if (s != cur) {
-                load_lane_x(xs, s, lane, &lx);
-                cur = s;
-            }
-            const bool ok = wait_bounded(full + slot, phase, P.ws, &abort_flag, lane);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            const int gs = pc.s0 + s;
-            const int bs = min(q4b::kSliceBlocks, nb - gs * q4b::kSliceBlocks);
-            const int nr = min(q4b::kTileRows, pc.r1 - pc.r0 - t * q4b::kTileRows);
-            const uint8_t* sb = ring + (size_t)slot * q4b::kSlotBytes;
-            float val[8];
-            if (!lx.flagged) {
-                const float ls = lx.scale;
-                if (kDMap && bs == q4b::kSliceBlocks && nr == q4b::kTileRows) {
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                        const uint32_t dh =
-                            *reinterpret_cast<const uint16_t*>(sb + q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane);
-                        val[r] = half_bits_f32(dh) * ls * block_dot16(q, lx.p);
-                    }
-                } else {
-                    q4b::Piece pp;
-                    pp.r0 = pc.r0;
-                    pp.r1 = pc.r1;
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                        const uint32_t dh = *reinterpret_cast<const uint16_t*>(
-                            sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
-                                        : q4b::scale_offset(G, pp, t, gs, r, lane)));
-                        const float dot = block_dot16(q, lx.p);
-                        val[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * ls * dot : 0.0f;
-                    }
-                }
-            } else {
-                // exact path: binary32 products with the activations themselves
-                q4b::Piece pp;
-                pp.r0 = pc.r0;
-                pp.r1 = pc.r1;
-                float4 xf[8];
-                const float4* xg = reinterpret_cast<const float4*>(G.x + ((int64_t)gs * q4b::kSliceBlocks + lane) * 32);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) xf[k] = lane < bs ? __ldcg(xg + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const uint4 q = *reinterpret_cast<const uint4*>(sb + r * (q4b::kSliceBlocks * 16) + lane * 16);
-                    const uint32_t dh = *reinterpret_cast<const uint16_t*>(
-                        sb + (kDMap ? q4b::kSlotQs + r * q4b::kDMapRow + 2 * lane
-                                    : q4b::scale_offset(G, pp, t, gs, r, lane)));
-                    const float2 d2 = block_dot(q, xf, kc);
-                    val[r] = (lane < bs && r < nr) ? half_bits_f32(dh) * (d2.x + d2.y) : 0.0f;
-                }
-            }
-            // the slot is read: refill it with unit v + slots, which may belong to a
-            // later group (the proxy fence orders this warp's shared-memory reads
-            // before the copies' writes)
-            __syncwarp();
-            if (rc.valid(P)) {
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                issue_stack_unit<kDMap>(P, rc, slot, ring, full, lane, (vr / q4s::kSWarps) & 31);
-                rc.advance(P, c);
-                vr += q4s::kSWarps;
-            }
-            const float row_sum = reduce8(val, lane);
-            const int r = lane >> 2;
-            if ((lane & 3) == 0 && r < nr) red[(t * q4b::kTileRows + r) * S + s] = row_sum;
-            cu.advance(dt, ds, S);
-            slot += q4s::kSWarps;
-            if (slot >= slots) {
-                slot -= slots;
-                phase ^= 1u;
-            }
-        }
-        __syncthreads();
-        if (*abort_v) break;
-
-        // each row's slices in slice order
-        const int rows = pc.r1 - pc.r0;
-        if (G.splits == 1) {
-            for (int i = tid; i < rows; i += q4s::kSThreads) {
-                float sum = 0.0f;
-                for (int k = 0; k < S; ++k) sum += red[i * S + k];
-                G.y[pc.r0 + i] = sum;
-            }
-        } else {
-            // K split: partial sums, then the row range's ticket; the piece that
-            // arrives last adds the partials in split order and resets the ticket
-            float* part = reinterpret_cast<float*>(P.ws) + G.part_off;
-            uint32_t* ticket = P.ws + G.ticket_off + pc.j;
-            for (int i = tid; i < rows; i += q4s::kSThreads) {
-                float sum = 0.0f;
-                for (int k = 0; k < S; ++k) sum += red[i * S + k];
-                part[(int64_t)pc.split * G.n + pc.r0 + i] = sum;
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) last_split = atomicAdd(ticket, 1u) == (uint32_t)G.splits - 1u;
-            __syncthreads();
-            if (last_split) {
-                __threadfence();
-                for (int i = tid; i < rows; i += q4s::kSThreads) {
-                    const int64_t row = pc.r0 + i;
-                    float sum = 0.0f;
-                    for (int sp = 0; sp < G.splits; ++sp) sum += __ldcg(part + (int64_t)sp * G.n + row);
-                    G.y[row] = sum;
-                }
-                if (tid == 0) *ticket = 0u;
-            }
-        }
-        // the piece's results are visible before its completion count
-        if (gi + 1 < P.ngroups) {
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicAdd(P.ws + P.grp[gi].counter, 1u);
-        }
-        base += U;
-    }
-    if (*abort_v) {
-        // leave no copy in flight: wait (bounded) for the units this warp
-        // requested and did not read
-        for (int u = v; u < vr; u += q4s::kSWarps) mbar_wait_short_bounded(full + u % slots, (uint32_t)(u / slots) & 1u);
-    }
-}
-
-namespace {
-cudaError_t setup_stack_kernel(int optin_smem) {
-    for (int i = 0; i < 2; ++i) {
-        const void* f = i ? (const void*)stack_b1_kernel<true> : (const void*)stack_b1_kernel<false>;
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, f);
-        if (e != cudaSuccess) return e;
-        if (q4s::kSmemBudget + (int)fa.sharedSizeBytes > optin_smem) return cudaErrorInvalidValue;
-        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, q4s::kSmemBudget);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-}  // namespace
-
-// One launch of the persistent stack kernel: one CTA per piece of the largest
-// group (at most one per SM, so that every CTA is resident at once).
-cudaError_t launch_stack_b1(const q4s::Params& P, int grid, bool pdl, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(q4s::kSThreads, 1, 1);
-    cfg.dynamicSmemBytes = q4s::smem_bytes(P);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    bool all_maps = true;
-    for (int i = 0; i < P.ngroups; ++i)
-        for (int k = P.grp[i].first; k < P.grp[i].first + P.grp[i].count; ++k) all_maps = all_maps && P.gemv[k].desc.d_map;
-    return all_maps ? cudaLaunchKernelEx(&cfg, stack_b1_kernel<true>, P)
-                    : cudaLaunchKernelEx(&cfg, stack_b1_kernel<false>, P);
-}
-
 namespace {
 template <int B>
 cudaError_t setup_b1_tokens(int optin_smem) {
@@ -842,8 +530,7 @@ cudaError_t setup_b1_tokens(int optin_smem) {
 }  // namespace
 
 cudaError_t setup_b1_kernel(int optin_smem) {
-    cudaError_t e = setup_stack_kernel(optin_smem);
-    if (e == cudaSuccess) e = setup_b1_tokens<1>(optin_smem);
+    cudaError_t e = setup_b1_tokens<1>(optin_smem);
     if (e == cudaSuccess) e = setup_b1_tokens<2>(optin_smem);
     if (e == cudaSuccess) e = setup_b1_tokens<3>(optin_smem);
     if (e == cudaSuccess) e = setup_b1_tokens<4>(optin_smem);

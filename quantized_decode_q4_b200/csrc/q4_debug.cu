@@ -4,7 +4,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <array>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -13,7 +12,6 @@
 #include "../../include/q4.h"
 #include "../../include/q4_debug.h"
 #include "q4_b1_plan.h"
-#include "q4_stack_plan.h"
 #include "q4_device.cuh"
 #include "q4_host.h"
 #include "q4_intdot.cuh"
@@ -182,167 +180,6 @@ int q4_debug_check_b1(const int64_t* n, const int64_t* k, int count, int b, int 
                 return 27;
         }
     }
-    return 0;
-}
-
-int q4_debug_check_stack(const int64_t* n, const int64_t* k, const int* group, int count, int num_sms,
-                         int64_t* launches) {
-    using namespace q4s;
-    if (!n || !k || !group || count < 1 || num_sms < 1) return 1;
-    // groups exactly as q4_layer_stack splits them
-    std::vector<std::pair<int, int>> groups;
-    int begin = 0;
-    for (int i = 1; i <= count; ++i) {
-        if (i < count && group[i] < group[i - 1]) return 1;
-        if (i == count || group[i] != group[i - 1]) {
-            if (i - begin > Q4_MAX_GROUP) return 1;
-            groups.push_back({begin, i});
-            begin = i;
-        }
-    }
-    std::vector<Shape> sh((size_t)count);
-    for (int i = 0; i < count; ++i) sh[i] = {n[i], k[i]};
-    // ticket words as stack_check sizes them: the largest group's, then one count per group
-    int64_t tmax = 0, pmax = 0;
-    for (auto& g : groups) {
-        int64_t t = 0, p = 0;
-        if (group_need(sh.data() + g.first, g.second - g.first, 1, num_sms, &t, &p) != Q4_OK) return 2;
-        tmax = std::max(tmax, t);
-        pmax = std::max(pmax, p);
-    }
-    const int64_t count_word = kHeaderBytes / 4 + tmax;
-    const int64_t tickets = tmax + (int64_t)groups.size();
-    const int64_t part_base = part_base_for(tickets);
-    if ((count_word + (int64_t)groups.size()) * 4 > part_base) return 3;
-    std::vector<Params> chunk(1);
-    int64_t nl = 0;
-    for (int g0 = 0; g0 < (int)groups.size();) {
-        int g1 = g0;
-        bool alone = false;
-        stack_chunk(sh.data(), groups, g0, num_sms, &g1, &alone);
-        if (g1 <= g0 || g1 - g0 > kStackGroups) return 4;
-        if (alone) {
-            // a group with more pieces than multiprocessors runs on its own
-            if (g1 != g0 + 1 || group_pieces(sh.data(), groups[g0], num_sms) <= num_sms) return 4;
-            ++nl;
-            g0 = g1;
-            continue;
-        }
-        int gemvs = 0;
-        for (int gi = g0; gi < g1; ++gi) {
-            gemvs += groups[gi].second - groups[gi].first;
-            if (group_pieces(sh.data(), groups[gi], num_sms) > num_sms) return 4;
-        }
-        if (gemvs > kStackGemvs) return 4;
-        // a chunk ends only where the next group would not fit
-        if (g1 < (int)groups.size() && g1 - g0 < kStackGroups &&
-            gemvs + (groups[g1].second - groups[g1].first) <= kStackGemvs &&
-            group_pieces(sh.data(), groups[g1], num_sms) <= num_sms)
-            return 4;
-        Params& P = chunk[0];
-        int grid = 0;
-        if (plan_stack(sh.data(), groups, g0, g1, part_base, count_word, num_sms, &P, &grid) != Q4_OK) return 5;
-        ++nl;
-        if (P.ngroups != g1 - g0) return 5;
-        if (smem_bytes(P) > (uint32_t)kSmemBudget) return 6;
-        if (P.slots < kSWarps || P.slots > kMaxSlots || P.slots % kSWarps) return 6;
-        if (ring_offset(P) % 128 || x_offset(P) % 16 || red_offset() % 16) return 6;
-        if (grid < 1 || grid > num_sms) return 7;
-        int maxp = 0;
-        for (int gi = 0; gi < P.ngroups; ++gi) {
-            const Group& G = P.grp[gi];
-            const int src = groups[g0 + gi].first;
-            if (G.count != groups[g0 + gi].second - src || G.npieces < 1) return 8;
-            if (G.counter != count_word + g0 + gi) return 8;
-            maxp = std::max(maxp, G.npieces);
-            // the group's GEMVs: the same plan as one launch of the group would use
-            q4b::Params B;
-            int64_t t = 0, e = 0;
-            if (plan_b1(sh.data() + src, G.count, 1, part_base, num_sms, &B, &t, &e) != Q4_OK) return 9;
-            if (B.npieces != G.npieces) return 9;
-            for (int i = 0; i < G.count; ++i) {
-                const q4b::Desc& D = P.gemv[G.first + i].desc;
-                if (D.n != sh[src + i].n || (int64_t)D.nb * 32 != sh[src + i].k) return 9;
-                if (D.piece_begin != B.g[i].piece_begin || D.splits != B.g[i].splits || D.cps != B.g[i].cps)
-                    return 9;
-                if (D.splits > 1 && ((D.ticket_off + D.n) * 4 > count_word * 4 || D.ticket_off * 4 < kHeaderBytes))
-                    return 9;  // tickets below the counts
-                if (D.splits > 1 && (D.part_off * 4 < part_base || (D.part_off + (int64_t)D.splits * D.n) * 4 >
-                                                                       part_base + pmax))
-                    return 9;
-            }
-        }
-        if (maxp != grid) return 7;
-        // every CTA: the pieces it takes, then each warp's requests and reads
-        for (int c = 0; c < grid; ++c) {
-            std::vector<std::vector<uint8_t>> seen(P.ngroups);
-            for (int gi = 0; gi < P.ngroups; ++gi) {
-                Piece pc;
-                if (!piece_of(P, gi, c, &pc)) continue;
-                const q4b::Desc& D = P.gemv[pc.gemv].desc;
-                if (pc.gemv < P.grp[gi].first || pc.gemv >= P.grp[gi].first + P.grp[gi].count) return 10;
-                if (pc.r0 < 0 || pc.r1 <= pc.r0 || pc.r1 > D.n) return 10;
-                if (pc.S < 1 || pc.S > q4b::kPieceSlices || pc.s0 + pc.S > D.nslices) return 11;
-                if ((uint32_t)pc.S * q4b::kXSliceBytes > P.x_bytes) return 11;
-                if (q4b::xchunk_offset(pc.S - 1, q4b::kXChunks - 1, q4b::kSliceBlocks - 1) + 16 > P.x_bytes) return 11;
-                if ((int64_t)pc.T * q4b::kTileRows * pc.S * 4 > (int64_t)P.red_bytes) return 11;
-                seen[gi].assign((size_t)pc.U, 0);
-            }
-            for (int w = 0; w < kSWarps; ++w) {
-                // requests: the sequence walked by Seq, into slot v % slots
-                std::vector<std::array<int, 3>> req;
-                Seq rc;
-                rc.start(P, c, w);
-                int vr = w;
-                for (; rc.valid(P); vr += kSWarps) {
-                    if (rc.gi < 0 || rc.gi >= P.ngroups) return 12;
-                    if (rc.t < 0 || rc.s < 0 || rc.s >= rc.p.S || rc.t * rc.p.S + rc.s != rc.lu || rc.lu >= rc.p.U)
-                        return 12;
-                    // 16-byte aligned tensor-map x coordinate inside the code row
-                    const int gsl = rc.p.s0 + rc.s;
-                    if ((gsl * q4b::kSliceBlocks * 16) % 16 || (int64_t)gsl * q4b::kSliceBlocks * 16 >=
-                                                                    (int64_t)P.gemv[rc.p.gemv].desc.nb * 16)
-                        return 12;
-                    req.push_back({rc.gi, rc.t, rc.s});
-                    rc.advance(P, c);
-                    if ((int64_t)req.size() > (int64_t(1) << 26)) return 12;
-                }
-                // reads: the kernel's group loop (base, v, the cursor's stepping)
-                int v = w, base = 0;
-                size_t r = 0;
-                for (int gi = 0; gi < P.ngroups; ++gi) {
-                    Piece pc;
-                    if (!piece_of(P, gi, c, &pc)) continue;
-                    if (v < base || v >= base + kSWarps) return 13;
-                    int t = (v - base) / pc.S, s = (v - base) - ((v - base) / pc.S) * pc.S;
-                    const int dt = kSWarps / pc.S, ds = kSWarps - dt * pc.S;
-                    for (; v < base + pc.U; v += kSWarps) {
-                        const int lu = v - base;
-                        if (t * pc.S + s != lu) return 13;
-                        // the unit read is the one requested into this slot
-                        if ((v - w) % kSWarps || r >= req.size()) return 14;
-                        if (req[r][0] != gi || req[r][1] != t || req[r][2] != s) return 14;
-                        ++r;
-                        if (seen[gi][(size_t)lu]) return 15;
-                        seen[gi][(size_t)lu] = 1;
-                        t += dt;
-                        s += ds;
-                        if (s >= pc.S) {
-                            s -= pc.S;
-                            ++t;
-                        }
-                    }
-                    base += pc.U;
-                }
-                if (r != req.size()) return 14;  // every request is read
-            }
-            for (int gi = 0; gi < P.ngroups; ++gi)
-                for (uint8_t x : seen[gi])
-                    if (!x) return 15;
-        }
-        g0 = g1;
-    }
-    if (launches) *launches = nl;
     return 0;
 }
 

@@ -9,7 +9,6 @@
 
 #include "../../include/q4.h"
 #include "q4_b1_plan.h"
-#include "q4_stack_plan.h"
 #include "q4_tc_plan.h"
 
 namespace q4k {
@@ -19,7 +18,6 @@ cudaError_t launch_dequant(const uint8_t* qs, const uint16_t* d, float* out, int
                            int num_sms, cudaStream_t stream);
 cudaError_t setup_b1_kernel(int optin_smem);
 cudaError_t launch_b1(const q4b::Params& P, bool pdl, cudaStream_t stream);
-cudaError_t launch_stack_b1(const q4s::Params& P, int grid, bool pdl, cudaStream_t stream);
 cudaError_t encode_b1_maps(CUtensorMap* qs_map, CUtensorMap* d_map, int32_t* d_ok, const uint8_t* qs,
                            const uint16_t* d, int64_t n, int64_t k);
 cudaError_t setup_tc_kernels(int optin_smem);
@@ -68,22 +66,6 @@ q4_status plan_b1(const Shape* sh, int count, int b, int64_t part_base, int num_
 // Tensor-core plan (q4b::kMaxTokens < b <= 16) of one launch; same outputs.
 q4_status plan_tc(const Shape* sh, int count, int b, int64_t part_base, int num_sms,
                   q4t::Params* P, int64_t* tickets, int64_t* ws_end);
-
-// One launch of the persistent batch-1 stack kernel over groups [g0, g1) of a
-// stack (index ranges into its GEMVs): every group planned as plan_b1 would
-// (one token), the completion count of group i at workspace word
-// count_word + i. Fills everything except the pointers and tensor maps when
-// `stack` is null (the shapes come from `sh`, one per GEMV of the stack).
-// *grid = CTAs of the launch.
-q4_status plan_stack(const Shape* sh, const std::vector<std::pair<int, int>>& groups, int g0, int g1,
-                     int64_t part_base, int64_t count_word, int num_sms, q4s::Params* P, int* grid);
-
-// Groups [g0, *g1) that one launch of the stack kernel takes, starting at g0;
-// *alone: group g0 alone (*g1 = g0 + 1) needs more pieces than the device has
-// multiprocessors and runs as a launch of the one-group kernel instead.
-void stack_chunk(const Shape* sh, const std::vector<std::pair<int, int>>& groups, int g0, int num_sms, int* g1,
-                 bool* alone);
-int group_pieces(const Shape* sh, const std::pair<int, int>& g, int num_sms);
 
 // Start of the partial sums for a ticket region of `tickets` words.
 int64_t part_base_for(int64_t tickets);

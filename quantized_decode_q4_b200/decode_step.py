@@ -73,17 +73,8 @@ class DecodeStep:
 
     @property
     def launches(self) -> int:
-        """Kernels one step launches. One token: the persistent stack kernel, each
-        launch over as many consecutive groups as its parameters hold (the
-        library's own plan, replayed on the host for this device's SM count).
-        2..16 tokens: one launch per dependency group."""
-        if self.batch == 1:
-            sms = torch.cuda.get_device_properties(self.device).multi_processor_count
-            shapes = [(g.n, g.k) for g in self.workload.gemvs]
-            st, n = q4.check_stack(shapes, self.groups, sms)
-            if st != 0:
-                raise RuntimeError(f"stack plan replay failed ({st})")
-            return n
+        """Kernels one step launches: one per dependency group (batch 1 on the CUDA
+        cores, 2..16 tokens on the tensor cores, all tokens in one launch)."""
         return self.workload.n_groups
 
     def weight_copies(self, r: int) -> list:

@@ -77,17 +77,14 @@ def test_8b_class_stack_full_size(b):
 
 @pytest.mark.parametrize("b", [1, 4])
 def test_step_launch_count(b):
-    """One token: the persistent stack kernel, three launches for the 121 groups
-    (each launch carries at most 80 GEMVs); more tokens: one kernel per dependency
-    group. The figure bench.py reports."""
+    """One kernel per dependency group, whatever the batch (the figure bench.py reports)."""
     step = DecodeStep(synth.workloads()["smollm2_135m"], b)
     step.run()
     torch.cuda.synchronize()
     c0 = q4.launch_count()
     step.run()
     torch.cuda.synchronize()
-    want = 3 if b == 1 else synth.workloads()["smollm2_135m"].n_groups
-    assert q4.launch_count() - c0 == step.launches == want
+    assert q4.launch_count() - c0 == step.launches == synth.workloads()["smollm2_135m"].n_groups
 
 
 def _chained_stack(d: int, f: int, layers: int, seed: int):
@@ -120,15 +117,14 @@ def _chained_stack(d: int, f: int, layers: int, seed: int):
 
 @pytest.mark.parametrize("d,f", [(1024, 2816), (960, 2560)])
 def test_chained_stack_waits_for_earlier_groups(d, f):
-    """Groups that read the outputs of the group before them, over 80 groups (two
-    launches of the persistent kernel): the step must give bit for bit the
-    outputs of the same groups enqueued one call each (stream order between every
-    group), in direct launches and graph replays; the first group, whose input is
-    synthetic, must also match the oracle."""
+    """Groups that read the outputs of the group before them, over 80 groups
+    (launches that start while the previous one drains, their weights streaming
+    in before they wait): the step must give bit for bit the outputs of the same
+    groups enqueued one call each, in direct launches and graph replays; the
+    first group, whose input is synthetic, must also match the oracle."""
     spec, mats, xs, ys = _chained_stack(d, f, 16, 31)
     groups = [s[2] for s in spec]
     stack = q4.Stack(mats, xs, ys, groups)
-    assert q4.check_stack([(s[0], s[1]) for s in spec], groups)[1] == 2
     ws = q4.workspace(stack.workspace_bytes(1), "cuda")
     q4.layer_stack(stack, 1, ws)
     torch.cuda.synchronize()

@@ -226,40 +226,3 @@ def test_interchange_matches_oracle():
     qs, d = q4.blocks_to_planes(blocks, n, k)
     assert np.array_equal(qs, qs_o) and np.array_equal(d, d_o)
     assert np.array_equal(q4.planes_to_blocks(qs, d, n, k), blocks)
-
-
-def _stack_of(wl):
-    return [(g.n, g.k) for g in wl.gemvs], [g.group for g in wl.gemvs]
-
-
-@pytest.mark.parametrize("num_sms", [148, 132, 7])
-def test_stack_plans_replay_on_host(num_sms):
-    """The persistent one-token stack kernel: every workload's step split into
-    launches that fit the kernel's parameters, one CTA per multiprocessor at
-    most, completion counts between tickets and partial sums, and every warp's
-    requests matching its reads unit for unit, across group boundaries."""
-    for name, wl in synth.workloads().items():
-        shapes, groups = _stack_of(wl)
-        st, launches = q4.check_stack(shapes, groups, num_sms)
-        assert st == 0, (name, num_sms, st)
-        assert 1 <= launches <= len(set(groups))
-    # the 8B-class step (224 GEMVs, 128 groups) fits three launches
-    shapes, groups = _stack_of(synth.workloads()["llama8b_class"])
-    assert q4.check_stack(shapes, groups, 148) == (0, 3)
-
-
-def test_stack_plans_replay_random():
-    """Seeded random stacks: groups of 1..8 GEMVs with ragged rows, K from one
-    block to 32768, tiny groups that leave most CTAs without a piece, and more
-    groups than one launch carries."""
-    rng = np.random.default_rng(11)
-    ns = [1, 3, 8, 17, 100, 147, 148, 149, 300, 1000, 4096]
-    kbs = [1, 3, 31, 32, 33, 100, 128, 129, 448, 1000]
-    for it in range(60):
-        shapes, groups = [], []
-        for gi in range(int(rng.integers(1, 90 if it % 10 == 0 else 12))):
-            for _ in range(int(rng.integers(1, 9))):
-                shapes.append((int(rng.choice(ns)), 32 * int(rng.choice(kbs))))
-                groups.append(gi)
-        st, _ = q4.check_stack(shapes, groups, int(rng.choice([148, 64, 9])))
-        assert st == 0, (it, st)
